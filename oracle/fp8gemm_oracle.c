@@ -1,0 +1,217 @@
+/*
+ * fp8gemm_oracle.c -- CPU oracle for the FP8 (e4m3) block-scaled NT GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, plain, obviously-correct
+ * definition that the CUDA library is checked against.  Only the tests, the
+ * smoke check and the benchmark's CPU-baseline leg load it.  It shares no code,
+ * header, table or constant with the CUDA library under moe_grouped_gemm_08_b200/.
+ *
+ * What it computes (sources, by page and section):
+ *   - "DeepGEMM" product page (flashmla.org), section "What is DeepGEMM":
+ *     an FP8 GEMM library with one normal (dense) layout and two MoE layouts,
+ *     contiguous and masked.
+ *   - "DeepGEMM" how-to (aisharenet.com), section "Main functions" 1-3:
+ *     gemm_fp8_fp8_bf16_nt, m_grouped_gemm_fp8_fp8_bf16_nt_contiguous and
+ *     m_grouped_gemm_fp8_fp8_bf16_nt_masked; FP8 inputs, BF16 output.
+ *   - "DeepGEMM: Efficienza e Precisione..." (turtlesai.it), summary paragraph:
+ *     NT layout only (LHS not transposed, RHS transposed), fine-grained
+ *     scaling, two-level accumulation on CUDA cores.
+ *   - DeepSeek DeepGEMM news article (senqingzn.com), optimisation paragraph:
+ *     the FP8 tensor-core accumulation is not precise enough, so partial sums
+ *     are promoted into a higher-precision accumulator.
+ * The pages leave the scale granularities open.  This oracle takes 1x128
+ * (one fp32 scale per row of A per 128-wide K block, stored column-major with
+ * leading dimension ld) and 128x128 (one fp32 scale per 128x128 block of B).
+ *
+ * Definition, for every output element:
+ *   S_kb   = sum_{k in block kb} dec(A[m,k]) * dec(B[n,k])        (fp64, exact)
+ *   C[m,n] = bf16_rne( sum_kb S_kb * (sfa[kb][m] * sfb[n/128][kb]) )  (fp64)
+ * Every e4m3 product is a multiple of 2^-18 below 2^18 in magnitude, so a sum
+ * of at most 128 of them needs fewer than 44 significant bits and S_kb is exact
+ * in fp64.  The product of two fp32 scales is exact in fp64 (48 bits).  The
+ * only roundings are the fp64 scale multiply, the fp64 accumulation over kb
+ * (in ascending kb order) and the single final rounding to bf16.
+ *
+ * Build: plain C11, -ffp-contract=off, OpenMP over output rows.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORC_BLOCK 128
+
+/* ---------------------------------------------------------------------------
+ * e4m3 ("fn" variant) decode table, built from the format definition:
+ * 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0
+ * encodes subnormals m/8 * 2^-6; S.1111.111 is NaN; there is no infinity, so
+ * the largest finite magnitude is 1.75 * 2^8 = 448.
+ * ------------------------------------------------------------------------- */
+static double g_dec[256];
+static int g_dec_ready = 0;
+
+static void build_decode_table(void) {
+    for (int code = 0; code < 256; ++code) {
+        int sign = (code >> 7) & 1;
+        int e = (code >> 3) & 0xF;
+        int m = code & 0x7;
+        double v;
+        if (e == 0xF && m == 0x7) {
+            v = NAN;
+        } else if (e == 0) {
+            v = ldexp((double)m / 8.0, -6);
+        } else {
+            v = ldexp(1.0 + (double)m / 8.0, e - 7);
+        }
+        g_dec[code] = sign ? -v : v;
+    }
+    g_dec_ready = 1;
+}
+
+static const double *dec_table(void) {
+    if (!g_dec_ready) build_decode_table();
+    return g_dec;
+}
+
+void oracle_e4m3_decode_table(double *out256) {
+    memcpy(out256, dec_table(), sizeof(double) * 256);
+}
+
+/* ---------------------------------------------------------------------------
+ * fp64 -> bf16 with one round-to-nearest-even step.
+ * bf16 = 1 sign, 8 exponent (bias 127), 7 mantissa bits: 8 significant bits
+ * for normals, a fixed quantum of 2^-133 below 2^-126, overflow to infinity.
+ * Output: the bf16 bit pattern.
+ * ------------------------------------------------------------------------- */
+uint16_t oracle_bf16_from_f64(double x) {
+    if (isnan(x)) return (uint16_t)(signbit(x) ? 0xFFC0u : 0x7FC0u);
+    if (isinf(x)) return (uint16_t)(signbit(x) ? 0xFF80u : 0x7F80u);
+    if (x == 0.0) return (uint16_t)(signbit(x) ? 0x8000u : 0x0000u);
+    int e;
+    (void)frexp(x, &e);            /* |x| in [2^(e-1), 2^e) */
+    int q = e - 8;                 /* quantum of an 8-significant-bit number */
+    if (q < -133) q = -133;        /* bf16 subnormal quantum */
+    double scaled = ldexp(x, -q);  /* exact: power-of-two rescale */
+    double r = nearbyint(scaled);  /* default rounding mode: to nearest, ties even */
+    double y = ldexp(r, q);
+    if (fabs(y) >= ldexp(1.0, 128)) return (uint16_t)(signbit(x) ? 0xFF80u : 0x7F80u);
+    float yf = (float)y;           /* exact: y has at most 8 significant bits */
+    uint32_t bits;
+    memcpy(&bits, &yf, sizeof bits);
+    return (uint16_t)(bits >> 16);
+}
+
+/* ---------------------------------------------------------------------------
+ * One output row of the dense NT product (the definition above).
+ *   a_row : K e4m3 codes of row m of A
+ *   sfa_m : sfa + m, stepping by ld between K blocks (column-major scales)
+ *   B     : N x K e4m3 codes, row-major
+ *   sfb   : ceil(N/128) x ceil(K/128) fp32, row-major
+ *   c_row : N bf16 outputs; acc_row (optional) receives the fp64 pre-rounding value
+ * ------------------------------------------------------------------------- */
+static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
+                   const uint8_t *B, const float *sfb, int N, int K,
+                   uint16_t *c_row, double *acc_row) {
+    const double *dec = dec_table();
+    const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
+    for (int n = 0; n < N; ++n) {
+        const uint8_t *b_row = B + (size_t)n * K;
+        double acc = 0.0;
+        for (int kb = 0; kb < KB; ++kb) {
+            int k0 = kb * ORC_BLOCK;
+            int k1 = k0 + ORC_BLOCK < K ? k0 + ORC_BLOCK : K;
+            double s = 0.0;
+            for (int k = k0; k < k1; ++k) s += dec[a_row[k]] * dec[b_row[k]];
+            double scale = (double)sfa_m[(size_t)kb * ld] *
+                           (double)sfb[(size_t)(n / ORC_BLOCK) * KB + kb];
+            acc += s * scale;
+        }
+        c_row[n] = oracle_bf16_from_f64(acc);
+        if (acc_row) acc_row[n] = acc;
+    }
+}
+
+/* Dense: C[M,N] = A[M,K] . B[N,K]^T with sfa[KB][ld] and sfb[NB][KB].
+ * acc (optional, M x N fp64) receives the unrounded values. */
+void oracle_gemm_nt(const uint8_t *A, const float *sfa, long ld,
+                    const uint8_t *B, const float *sfb,
+                    int M, int N, int K, uint16_t *C, double *acc) {
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int m = 0; m < M; ++m)
+        row_nt(A + (size_t)m * K, sfa + m, ld, B, sfb, N, K,
+               C + (size_t)m * N, acc ? acc + (size_t)m * N : NULL);
+}
+
+/* Dense, selected rows only: row rows[i] of the product goes to C[i,:].
+ * Used to check large products on a sample of rows. */
+void oracle_gemm_nt_rows(const uint8_t *A, const float *sfa, long ld,
+                         const uint8_t *B, const float *sfb,
+                         int M, int N, int K, const int *rows, int nrows,
+                         uint16_t *C, double *acc) {
+    (void)M;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < nrows; ++i) {
+        int m = rows[i];
+        row_nt(A + (size_t)m * K, sfa + m, ld, B, sfb, N, K,
+               C + (size_t)i * N, acc ? acc + (size_t)i * N : NULL);
+    }
+}
+
+/* M-grouped contiguous layout ("DeepGEMM" how-to, aisharenet.com, "Main
+ * functions" 2; news article, senqingzn.com, MoE-layout paragraph): the rows
+ * of all experts are concatenated along M; m_indices[m] names the expert of
+ * row m, or is -1 for a padding row.  Row m uses B[g] (N x K) and sfb[g].
+ * Rows whose index is -1 (or outside [0,G)) are not written.
+ * rows/nrows: optional subset (NULL = all M_total rows, C indexed by m).
+ * With a subset, row rows[i] goes to C[i,:]. */
+void oracle_grouped_contiguous(const uint8_t *A, const float *sfa, long ld,
+                               const uint8_t *B, const float *sfb,
+                               const int *m_indices, int M_total, int G,
+                               int N, int K, const int *rows, int nrows,
+                               uint16_t *C, double *acc) {
+    const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
+    const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
+    int count = rows ? nrows : M_total;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < count; ++i) {
+        int m = rows ? rows[i] : i;
+        int g = m_indices[m];
+        if (g < 0 || g >= G) continue;
+        row_nt(A + (size_t)m * K, sfa + m, ld,
+               B + (size_t)g * N * K, sfb + (size_t)g * NB * KB, N, K,
+               C + (size_t)i * N, acc ? acc + (size_t)i * N : NULL);
+    }
+}
+
+/* M-grouped masked layout ("DeepGEMM" how-to, aisharenet.com, "Main functions"
+ * 3; news article, senqingzn.com, decode paragraph): A is [G][Mmax][K],
+ * sfa is [G][KB][ld], C is [G][Mmax][N]; group g has masked_m[g] valid rows,
+ * which use B[g] and sfb[g].  Rows at or past masked_m[g] are not written. */
+void oracle_grouped_masked(const uint8_t *A, const float *sfa, long ld,
+                           const uint8_t *B, const float *sfb,
+                           const int *masked_m, int G, int Mmax, int N, int K,
+                           uint16_t *C, double *acc) {
+    const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
+    const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
+    long total = (long)G * Mmax;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (long gm = 0; gm < total; ++gm) {
+        int g = (int)(gm / Mmax);
+        int m = (int)(gm % Mmax);
+        int valid = masked_m[g];
+        if (valid > Mmax) valid = Mmax;
+        if (m >= valid) continue;
+        row_nt(A + ((size_t)g * Mmax + m) * K, sfa + (size_t)g * KB * ld + m, ld,
+               B + (size_t)g * N * K, sfb + (size_t)g * NB * KB, N, K,
+               C + ((size_t)g * Mmax + m) * N,
+               acc ? acc + ((size_t)g * Mmax + m) * N : NULL);
+    }
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
