@@ -1,0 +1,125 @@
+/*
+ * fp8gemm.h -- C ABI of the B200 (sm_100a) FP8 block-scaled NT GEMM library.
+ *
+ * The operation (all three entry points):
+ *   C[m, n] = bf16( sum_kb  P_kb[m, n] * sfa[kb][m] * sfb[n / 128][kb] ),
+ *   P_kb[m, n] = sum over the 128-wide K block kb of A[m, k] * B[n, k],
+ * with A and B in FP8 e4m3, P_kb computed by the tensor cores and promoted into
+ * FP32 accumulators once per K block ("two-level accumulation").
+ * Sources:
+ *   - "DeepGEMM" how-to (aisharenet.com), "Main functions" 1-3: the dense
+ *     gemm_fp8_fp8_bf16_nt and the M-grouped contiguous / masked GEMMs, FP8 in,
+ *     BF16 out, only M grouped, experts sharing N and K;
+ *   - "DeepGEMM: Efficienza e Precisione..." (turtlesai.it): NT layout only
+ *     (LHS not transposed, RHS transposed), fine-grained scaling, LHS scales
+ *     laid out for aligned TMA loads, two-level accumulation;
+ *   - DeepSeek DeepGEMM news article (senqingzn.com), optimisation and layout
+ *     paragraphs: promotion of FP8 tensor-core sums, contiguous layout for
+ *     prefill / training, masked layout for decode with unknown expert counts;
+ *   - "DeepGEMM" product page (flashmla.org), performance section: the masked
+ *     layout is usable under CUDA graphs.
+ * The pages leave the scale granularity open; this library fixes it to 1x128
+ * for A and 128x128 for B.
+ *
+ * Layouts (row-major unless stated, all pointers are DEVICE pointers):
+ *   A    : e4m3 codes, [M, K] (dense / contiguous) or [G, Mmax, K] (masked).
+ *   sfa  : fp32, column-major per K block: element (m, kb) at sfa[kb * ld + m],
+ *          ld = fg_sfa_ld(M) (dense / contiguous: M = all rows);
+ *          masked: [G][ceil(K/128)][fg_sfa_ld(Mmax)].
+ *   B    : e4m3 codes, [N, K] (dense) or [G, N, K] (grouped).
+ *   sfb  : fp32, [ceil(N/128), ceil(K/128)] (dense) or [G, ceil(N/128), ceil(K/128)].
+ *   C    : bf16, [M, N] (dense / contiguous) or [G, Mmax, N] (masked).
+ * Requirements: K % 16 == 0 and N % 8 == 0 (16-byte row strides); A, B, C
+ * 16-byte aligned; sfa, sfb 4-byte aligned; K may end in a partial block.
+ *
+ * Ownership: the caller owns every buffer.  The library allocates only in
+ * fg_init (a status word, a split-K workspace and its counters), never inside
+ * a GEMM call, so calls can be captured into CUDA graphs.  The workspace is
+ * per device; GEMM calls that use it must not run concurrently on different
+ * streams of the same device.
+ *
+ * Errors: every entry point returns a status code and never throws.  Argument
+ * errors are found on the host before any launch and launch nothing.  A device
+ * wait that times out (about two seconds) makes the kernel exit early and sets
+ * the device status word, read and cleared by fg_get_device_status().
+ */
+#ifndef FP8GEMM_H
+#define FP8GEMM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FG_OK = 0,
+  FG_ERR_INVALID_ARG = 1,     /* null pointer, negative or inconsistent size */
+  FG_ERR_ALIGNMENT = 2,       /* K % 16, N % 8 or a base pointer misaligned */
+  FG_ERR_UNSUPPORTED = 3,     /* valid but outside what this build supports (e.g. G > 1024) */
+  FG_ERR_NOT_INITIALIZED = 4, /* fg_init was not called for the current device */
+  FG_ERR_CUDA = 5,            /* a CUDA runtime / driver call failed */
+  FG_ERR_TIMEOUT = 6          /* a device-side wait ran out; the kernel exited early */
+} fg_status;
+
+/* Prepare the library on `device` (makes it current): queries the SM count,
+ * resolves the tensor-map encoder and allocates the status word, the split-K
+ * workspace and counters.  Idempotent.  Call it outside any stream capture. */
+fg_status fg_init(int device);
+
+/* Free everything fg_init allocated, on every device it was called for. */
+void fg_shutdown(void);
+
+/* Row alignment that each expert's rows must be padded to in the contiguous
+ * layout (the block size along M; cf. get_m_alignment_for_contiguous_layout in
+ * the aisharenet.com how-to, "Main functions" 2). */
+int fg_m_alignment(void);
+
+/* Leading dimension of the column-major A scales for M rows: M rounded up to a
+ * multiple of 4, so every K-block column starts on a 16-byte boundary. */
+int fg_sfa_ld(int M);
+
+/* Dense C[M,N] = A[M,K] . B[N,K]^T (gemm_fp8_fp8_bf16_nt).  M == 0 is a no-op.
+ * stream: a cudaStream_t (NULL = legacy default stream). */
+fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                      int M, int N, int K, void* stream);
+
+/* M-grouped contiguous (m_grouped_gemm_fp8_fp8_bf16_nt_contiguous):
+ * rows of all experts concatenated along M; m_indices[m] (device, int32) is the
+ * expert of row m or -1 for a padding row.  Each expert's rows start at a
+ * multiple of fg_m_alignment().  Row m uses B[g] and sfb[g]; padding rows and
+ * whole padding blocks are not written.  Indices >= G are treated as -1. */
+fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const void* B, const float* sfb,
+                                      void* C, const int* m_indices, int M_total, int G, int N, int K,
+                                      void* stream);
+
+/* M-grouped masked (m_grouped_gemm_fp8_fp8_bf16_nt_masked): group g owns rows
+ * [0, masked_m[g]) of A[g]; masked_m lives in DEVICE memory and is never read
+ * by the host, so the launch has a fixed shape and can be captured in a CUDA
+ * graph and replayed with new counts.  Rows at or past masked_m[g] of C[g] are
+ * left untouched; counts above Mmax are clamped to Mmax. */
+fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb,
+                                  void* C, const int* masked_m, int G, int Mmax, int N, int K,
+                                  void* stream);
+
+/* Synchronise `stream`, then read and clear the device status word:
+ * FG_OK, or FG_ERR_TIMEOUT if some kernel since the last call gave up a wait. */
+fg_status fg_get_device_status(void* stream);
+
+/* Human-readable name of a status code (static storage). */
+const char* fg_status_string(fg_status status);
+
+/* Dense-path selection, process-wide: 0 = automatic (M <= 128 takes the
+ * swap-AB stream-K kernel, larger M the tiled kernel), 1 = always tiled,
+ * 2 = always swap-AB stream-K (requires M <= 128).  Returns the previous value;
+ * an unknown value is ignored. */
+int fg_set_dense_path(int path);
+
+/* Number of GEMM kernel launches the library has issued in this process. */
+uint64_t fg_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8GEMM_H */

@@ -1,0 +1,189 @@
+"""Python binding of the B200 FP8 block-scaled NT GEMM library (libfp8gemm.so).
+
+Argument marshalling only: every step of the GEMM runs in the CUDA kernels of the
+library.  PyTorch supplies device memory and the current stream.  If the compiled
+library is missing, importing this package raises -- there is no fallback path.
+
+Entry points (names after the DeepGEMM how-to, aisharenet.com, "Main functions"):
+  gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None)
+  m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None)
+  m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None)
+  get_m_alignment_for_contiguous_layout(), sfa_ld(M)
+Layouts: A [M,K] / [G,Mmax,K] e4m3 (uint8 or float8_e4m3fn); sfa fp32 column-major
+per K block, [KB, sfa_ld(M)] / [G, KB, sfa_ld(Mmax)]; B [N,K] / [G,N,K]; sfb fp32
+[NB, KB] / [G, NB, KB]; C bf16 [M,N] / [G,Mmax,N].  See include/fp8gemm.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import pathlib
+
+import torch
+
+_HERE = pathlib.Path(__file__).resolve().parent
+LIB_PATH = _HERE / "libfp8gemm.so"
+
+if not LIB_PATH.exists():
+    raise ImportError(f"{LIB_PATH} is not built; run `python moe_grouped_gemm_08_b200/build.py` "
+                      "or __graft_entry__.build()")
+
+_lib = ctypes.CDLL(str(LIB_PATH))
+_vp, _int = ctypes.c_void_p, ctypes.c_int
+_lib.fg_init.argtypes = [_int]
+_lib.fg_init.restype = _int
+_lib.fg_shutdown.argtypes = []
+_lib.fg_shutdown.restype = None
+_lib.fg_m_alignment.restype = _int
+_lib.fg_sfa_ld.argtypes = [_int]
+_lib.fg_sfa_ld.restype = _int
+_lib.fp8_gemm_nt.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
+_lib.fp8_gemm_nt.restype = _int
+_lib.fp8_gemm_grouped_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
+_lib.fp8_gemm_grouped_contiguous.restype = _int
+_lib.fp8_gemm_grouped_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
+_lib.fp8_gemm_grouped_masked.restype = _int
+_lib.fg_get_device_status.argtypes = [_vp]
+_lib.fg_get_device_status.restype = _int
+_lib.fg_status_string.argtypes = [_int]
+_lib.fg_status_string.restype = ctypes.c_char_p
+_lib.fg_set_dense_path.argtypes = [_int]
+_lib.fg_set_dense_path.restype = _int
+_lib.fg_launch_count.argtypes = []
+_lib.fg_launch_count.restype = ctypes.c_uint64
+
+FG_OK = 0
+STATUS_NAMES = {i: _lib.fg_status_string(i).decode() for i in range(7)}
+lib = _lib  # the raw C ABI, for callers that marshal pointers themselves
+
+
+class FP8GemmError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+def _check(code: int, what: str) -> None:
+    if code != FG_OK:
+        raise FP8GemmError(code, what)
+
+
+_initialised: set[int] = set()
+
+
+def init(device: int | None = None) -> None:
+    dev = torch.cuda.current_device() if device is None else int(device)
+    if dev not in _initialised:
+        _check(_lib.fg_init(dev), "fg_init")
+        _initialised.add(dev)
+
+
+def get_m_alignment_for_contiguous_layout() -> int:
+    return int(_lib.fg_m_alignment())
+
+
+def sfa_ld(m: int) -> int:
+    return int(_lib.fg_sfa_ld(int(m)))
+
+
+def set_dense_path(path: int) -> int:
+    """0 automatic, 1 tiled kernel, 2 swap-AB stream-K kernel (M <= 128). Returns the old value."""
+    return int(_lib.fg_set_dense_path(int(path)))
+
+
+def launch_count() -> int:
+    return int(_lib.fg_launch_count())
+
+
+def device_status(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(_lib.fg_get_device_status(ctypes.c_void_p(s.cuda_stream)))
+
+
+def _bytes(t: torch.Tensor, what: str) -> torch.Tensor:
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError(f"{what} must be uint8 e4m3 codes or float8_e4m3fn, got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{what} must be a contiguous CUDA tensor")
+    return t
+
+
+def _f32(t: torch.Tensor, what: str) -> torch.Tensor:
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{what} must be a contiguous CUDA float32 tensor")
+    return t
+
+
+def _i32(t: torch.Tensor, what: str) -> torch.Tensor:
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{what} must be a contiguous CUDA int32 tensor")
+    return t
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _out(C, shape, device):
+    if C is None:
+        return torch.empty(shape, dtype=torch.bfloat16, device=device)
+    if C.dtype != torch.bfloat16 or tuple(C.shape) != tuple(shape) or not C.is_contiguous():
+        raise ValueError(f"C must be a contiguous bfloat16 tensor of shape {tuple(shape)}")
+    return C
+
+
+def _cdiv(a, b):
+    return (a + b - 1) // b
+
+
+def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None):
+    """Dense C[M,N] = A[M,K] . B[N,K]^T with 1x128 (A) and 128x128 (B) fp32 scales."""
+    A, B = _bytes(A, "A"), _bytes(B, "B")
+    sfa, sfb = _f32(sfa, "sfa"), _f32(sfb, "sfb")
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K or tuple(sfa.shape) != (_cdiv(K, 128), sfa_ld(M)) or \
+            tuple(sfb.shape) != (_cdiv(N, 128), _cdiv(K, 128)):
+        raise ValueError("inconsistent shapes")
+    C = _out(C, (M, N), A.device)
+    init(A.device.index)
+    _check(_lib.fp8_gemm_nt(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
+                            M, N, K, _stream(stream)), "fp8_gemm_nt")
+    return C
+
+
+def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None, stream=None):
+    """M-grouped contiguous: A[M_total,K], B[G,N,K], m_indices[M_total] (-1 = padding)."""
+    A, B = _bytes(A, "A"), _bytes(B, "B")
+    sfa, sfb, m_indices = _f32(sfa, "sfa"), _f32(sfb, "sfb"), _i32(m_indices, "m_indices")
+    M, K = A.shape
+    G, N = B.shape[0], B.shape[1]
+    if B.shape[2] != K or m_indices.numel() != M or tuple(sfa.shape) != (_cdiv(K, 128), sfa_ld(M)) or \
+            tuple(sfb.shape) != (G, _cdiv(N, 128), _cdiv(K, 128)):
+        raise ValueError("inconsistent shapes")
+    C = _out(C, (M, N), A.device)
+    init(A.device.index)
+    _check(_lib.fp8_gemm_grouped_contiguous(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                            C.data_ptr(), m_indices.data_ptr(), M, G, N, K, _stream(stream)),
+           "fp8_gemm_grouped_contiguous")
+    return C
+
+
+def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stream=None):
+    """M-grouped masked: A[G,Mmax,K], masked_m[G] on the device; rows >= masked_m[g] untouched."""
+    A, B = _bytes(A, "A"), _bytes(B, "B")
+    sfa, sfb, masked_m = _f32(sfa, "sfa"), _f32(sfb, "sfb"), _i32(masked_m, "masked_m")
+    G, Mmax, K = A.shape
+    N = B.shape[1]
+    if B.shape[0] != G or B.shape[2] != K or masked_m.numel() != G or \
+            tuple(sfa.shape) != (G, _cdiv(K, 128), sfa_ld(Mmax)) or \
+            tuple(sfb.shape) != (G, _cdiv(N, 128), _cdiv(K, 128)):
+        raise ValueError("inconsistent shapes")
+    C = _out(C, (G, Mmax, N), A.device)
+    init(A.device.index)
+    _check(_lib.fp8_gemm_grouped_masked(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                        C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, _stream(stream)),
+           "fp8_gemm_grouped_masked")
+    return C

@@ -1,0 +1,44 @@
+"""Build the sm_100a CUDA library in-tree (nvcc, no JIT): libfp8gemm.so next to this file."""
+from __future__ import annotations
+
+import os
+import pathlib
+import subprocess
+
+HERE = pathlib.Path(__file__).resolve().parent
+ROOT = HERE.parent
+SO = HERE / "libfp8gemm.so"
+SOURCES = [HERE / "csrc" / "fp8gemm_api.cu"]
+DEPENDS = SOURCES + [HERE / "csrc" / "fp8_gemm_kernels.cuh", HERE / "csrc" / "sm100_ptx.cuh",
+                     ROOT / "include" / "fp8gemm.h"]
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-shared", "-Xcompiler", "-fPIC",
+]
+
+
+def nvcc() -> str:
+    cand = os.path.join(os.environ.get("CUDA_HOME", "/usr/local/cuda"), "bin", "nvcc")
+    return cand if os.path.exists(cand) else "nvcc"
+
+
+def build(force: bool = False, verbose: bool = False) -> pathlib.Path:
+    """Compile the library if any source is newer than the built .so."""
+    if not force and SO.exists():
+        newest = max(p.stat().st_mtime for p in DEPENDS)
+        if SO.stat().st_mtime >= newest:
+            return SO
+    tmp = SO.with_suffix(".so.tmp%d" % os.getpid())
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", str(ROOT / "include"), "-I", str(HERE / "csrc"),
+           *(str(s) for s in SOURCES), "-o", str(tmp)]
+    if verbose:
+        cmd.insert(1, "-Xptxas=-v")
+    subprocess.check_call(cmd)
+    os.replace(tmp, SO)
+    return SO
+
+
+if __name__ == "__main__":
+    print(build(force=True, verbose=True))

@@ -1,0 +1,630 @@
+// fp8_gemm_kernels.cuh -- sm_100a kernels of the FP8 block-scaled NT GEMM.
+//
+// What they compute (see include/fp8gemm.h for the sources on the pages):
+//   C[m,n] = bf16( sum_kb P_kb[m,n] * sfa[kb][m] * sfb[n/128][kb] ),
+// P_kb = the 128-deep FP8 product of K block kb, formed by tcgen05.mma in TMEM
+// and promoted by CUDA-core warps into FP32 register accumulators (the
+// two-level accumulation of the news article's optimisation paragraph and of
+// the turtlesai.it summary).
+//
+// Both kernels use the same warp roles (320 threads):
+//   warps 0-7 : promotion + epilogue.  Warp w reads TMEM lanes 32*(w%4)..+31
+//               (the lane quadrant its SM sub-partition can reach) and column
+//               half w/4 of every partial tile.
+//   warp 8    : TMA producer (one elected lane): A/B K-block tiles into an
+//               S-stage shared-memory ring, 128-byte swizzled.
+//   warp 9    : TMEM owner and MMA issuer (one lane): per K block, four
+//               tcgen05.mma (K = 32 each) into a free TMEM partial buffer, then
+//               tcgen05.commit to release the smem stage and to hand the
+//               buffer to the promotion warps.
+// TMEM holds several partial buffers so the MMA of block kb+1.. runs while
+// block kb is being promoted; the FP32 accumulators live in registers.
+//
+// Kernel 1, fp8_gemm_tiled_kernel: persistent CTAs walk 128 x BN output tiles
+//   (dense, M-grouped contiguous, M-grouped masked), m-block fastest.  The
+//   masked walk enumerates only live tiles from masked_m read on the device.
+// Kernel 2, fp8_gemm_swap_streamk_kernel (dense, M <= 128, the decode shapes):
+//   swap-AB -- 128 weight rows of B form the MMA's M side and the MP tokens
+//   its N side -- and stream-K: the (n-block, K-block) units are split evenly
+//   over the persistent CTAs; tiles split between CTAs are summed by the last
+//   CTA to finish (fp32 partials in a workspace, fixed summation order, no
+//   CTA waits on another).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace fg {
+
+constexpr int kBlockK = 128;       // K block = scale granularity = one 128-byte swizzle row
+constexpr int kBlockM = 128;       // MMA M (rows of the TMEM accumulator)
+constexpr int kThreads = 320;
+constexpr int kPromoWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, far above any legal wait
+constexpr int kErrTimeout = 6;       // FG_ERR_TIMEOUT
+constexpr int kMaskedMaxGroups = 1024;
+
+enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
+
+struct TiledParams {
+  const float* sfa;
+  const float* sfb;
+  __nv_bfloat16* C;
+  const int* m_indices;  // contiguous
+  const int* masked_m;   // masked
+  int* status;
+  int M;        // dense: M, contiguous: M_total, masked: Mmax
+  int N;
+  int K;
+  int G;
+  int ld;       // sfa leading dimension
+  int num_kb;   // ceil(K / 128)
+  int num_nb;   // ceil(N / 128): sfb blocks per group
+  int m_blocks; // ceil(M / 128)
+  int n_blocks; // ceil(N / BN)
+};
+
+struct SwapParams {
+  const float* sfa;
+  const float* sfb;
+  __nv_bfloat16* C;
+  float* ws;       // 2 * gridDim.x partial tiles of MP x 128 fp32
+  int* counters;   // one per n-tile, zero between launches
+  int* status;
+  int M, N, K, ld;
+  int num_kb;
+  int n_tiles;     // ceil(N / 128)
+};
+
+__device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
+  const uint32_t a = smem_addr(p);
+  return p + ((1024u - (a & 1023u)) & 1023u);
+}
+
+__device__ __forceinline__ void report_timeout(int* status) { atomicCAS(status, 0, kErrTimeout); }
+
+// Wait for the phase of `bar` with parity `parity` regardless of the abort flag
+// (used only to drain this CTA's own copies after an abort); bounded.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// Bounded barrier of the promotion threads: each arrives on `bar` (count =
+// number of promotion threads) and waits for the phase to complete.  Unlike
+// bar.sync it gives up after the wait limit, so an aborting warp cannot leave
+// the others stuck.
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volatile int* abort_flag) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, abort_flag, kWaitLimitNs);
+  phase ^= 1u;
+  return ok;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// ============================================================================
+// Kernel 1: tiled (dense / contiguous / masked)
+// ============================================================================
+struct TileInfo {
+  int live;
+  int g;       // group (0 for dense)
+  int m0;      // first row of the tile within its row space (masked: within group g)
+  int n0;
+};
+
+template <int MODE>
+__device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* s_prefix, int live_mblocks, int t,
+                                               int BN) {
+  TileInfo ti;
+  if (MODE == kMasked) {
+    const int nb = t / live_mblocks;
+    const int lm = t - nb * live_mblocks;
+    int lo = 0, hi = p.G;  // largest g with s_prefix[g] <= lm
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_prefix[mid] <= lm) lo = mid; else hi = mid;
+    }
+    ti.live = 1;
+    ti.g = lo;
+    ti.m0 = (lm - s_prefix[lo]) * kBlockM;
+    ti.n0 = nb * BN;
+  } else {
+    const int nb = t / p.m_blocks;
+    const int mb = t - nb * p.m_blocks;
+    ti.m0 = mb * kBlockM;
+    ti.n0 = nb * BN;
+    if (MODE == kContiguous) {
+      const int g = __ldg(p.m_indices + ti.m0);
+      ti.live = (g >= 0 && g < p.G);
+      ti.g = ti.live ? g : 0;
+    } else {
+      ti.live = 1;
+      ti.g = 0;
+    }
+  }
+  return ti;
+}
+
+template <int BN, int STAGES, int NUM_TBUF, int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const TiledParams p) {
+  static_assert(BN == 128 || BN == 256, "BN");
+  constexpr int A_BYTES = kBlockM * kBlockK;
+  constexpr int B_BYTES = BN * kBlockK;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = NUM_TBUF * BN;
+  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+  constexpr int COLS = BN / 2;  // columns per promotion thread
+  constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + NUM_TBUF;
+  uint64_t* mma_done = tempty + NUM_TBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
+  if (warp == kMmaWarp) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+  if (MODE == kMasked && warp == 0) {
+    // live 128-row blocks per group, exclusive prefix in s_prefix[0..G]
+    int carry = 0;
+    if (lane == 0) s_prefix[0] = 0;
+    for (int base = 0; base < p.G; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < p.G) {
+        int cnt = __ldg(p.masked_m + g);
+        cnt = cnt < 0 ? 0 : (cnt > p.M ? p.M : cnt);
+        v = (cnt + kBlockM - 1) / kBlockM;
+      }
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (g < p.G) s_prefix[g + 1] = carry + v;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  int num_tiles, live_mblocks = 1;
+  if (MODE == kMasked) {
+    live_mblocks = s_prefix[p.G];
+    num_tiles = live_mblocks * p.n_blocks;
+  } else {
+    num_tiles = p.m_blocks * p.n_blocks;
+  }
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint64_t issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+        if (!ti.live) continue;
+        const int ga = (MODE == kMasked) ? ti.g : 0;
+        const int gb = (MODE == kDense) ? 0 : ti.g;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_3d(sa, &tmA, &full[stage], kb * kBlockK, ti.m0, ga);
+          tma_load_3d(sa + A_BYTES, &tmB, &full[stage], kb * kBlockK, ti.n0, gb);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {  // drain this CTA's copies still in flight before the CTA exits
+        const uint64_t first = issued > STAGES ? issued - STAGES : 0;
+        for (uint64_t i = first; i < issued; ++i)
+          mbar_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+        if (!ti.live) continue;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + tb * BN;
+          const uint32_t sa = smem_addr(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = smem_desc_k128_sw128(sa);
+          const uint64_t bdesc = smem_desc_k128_sw128(sa + A_BYTES);
+#pragma unroll
+          for (int j = 0; j < kBlockK / 32; ++j)  // 32 e4m3 = 32 bytes = 2 descriptor units per step
+            mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          mma_commit(&tfull[tb]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+        }
+      }
+      // every MMA this thread issued has finished once mma_done flips
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------ promotion + epilogue
+    const int q = warp & 3;
+    const int h = warp >> 2;
+    const int row = q * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t tb = 0, tphase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+      if (!ti.live) continue;
+      const int m = ti.m0 + row;
+      int row_limit;                 // rows of this tile's row space that exist
+      const float* sa_ptr;
+      if (MODE == kMasked) {
+        row_limit = p.M;
+        sa_ptr = p.sfa + static_cast<size_t>(ti.g) * p.num_kb * p.ld + m;
+      } else {
+        row_limit = p.M;
+        sa_ptr = p.sfa + m;
+      }
+      const bool row_ok = m < row_limit;
+      const int nb = (ti.n0 + h * COLS) / kBlockK;
+      const float* sb_ptr = p.sfb + (static_cast<size_t>(MODE == kDense ? 0 : ti.g) * p.num_nb + nb) * p.num_kb;
+
+      float acc[COLS];
+#pragma unroll
+      for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+
+      float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
+      float sb_next = __ldg(sb_ptr);
+      for (int kb = 0; kb < p.num_kb; ++kb) {
+        const float sa = sa_next, sb = sb_next;
+        if (kb + 1 < p.num_kb) {
+          sa_next = row_ok ? __ldg(sa_ptr + static_cast<size_t>(kb + 1) * p.ld) : 0.0f;
+          sb_next = __ldg(sb_ptr + kb + 1);
+        }
+        if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const float s = sa * sb;
+        const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
+#pragma unroll
+        for (int c0 = 0; c0 < COLS; c0 += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(taddr + c0, v0);
+          tmem_ld_32x32b_x32(taddr + c0 + 32, v1);
+          tmem_wait_ld();
+          if (c0 + 64 >= COLS) {  // whole slice read: hand the TMEM buffer back to the MMA
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[tb]);
+          }
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            acc[c0 + j] = fmaf(__uint_as_float(v0[j]), s, acc[c0 + j]);
+            acc[c0 + 32 + j] = fmaf(__uint_as_float(v1[j]), s, acc[c0 + 32 + j]);
+          }
+        }
+        if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+      }
+      if (!ok) break;
+
+      // epilogue: bf16 round-to-nearest-even, 16-byte stores of this thread's row segment
+      bool store_row = row_ok;
+      __nv_bfloat16* crow;
+      if (MODE == kMasked) {
+        int cnt = __ldg(p.masked_m + ti.g);
+        cnt = cnt > p.M ? p.M : cnt;
+        store_row = m < cnt;
+        crow = p.C + (static_cast<size_t>(ti.g) * p.M + m) * p.N;
+      } else {
+        if (MODE == kContiguous && store_row) store_row = __ldg(p.m_indices + m) == ti.g;
+        crow = p.C + static_cast<size_t>(m) * p.N;
+      }
+      if (store_row) {
+        const int nbase = ti.n0 + h * COLS;
+#pragma unroll
+        for (int j = 0; j < COLS; j += 8) {
+          if (nbase + j < p.N) {
+            uint4 v;
+            v.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
+            v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
+            v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
+            v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+            *reinterpret_cast<uint4*>(crow + nbase + j) = v;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status);
+}
+
+// ============================================================================
+// Kernel 2: swap-AB stream-K (dense, M <= MP <= 128)
+// ============================================================================
+__device__ __forceinline__ int sk_owner(long long u, int P, long long U) {
+  return static_cast<int>(((u + 1) * P - 1) / U);
+}
+__device__ __forceinline__ long long sk_begin(int c, int P, long long U) { return (c * U) / P; }
+
+template <int MP, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    fp8_gemm_swap_streamk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
+                                 const SwapParams p) {
+  static_assert(MP == 32 || MP == 64 || MP == 128, "MP");
+  constexpr int W_BYTES = kBlockM * kBlockK;  // 128 weight rows
+  constexpr int T_BYTES = MP * kBlockK;       // MP token rows
+  constexpr int STAGE_BYTES = W_BYTES + T_BYTES;
+  constexpr int NUM_TBUF = 4;
+  constexpr uint32_t TMEM_COLS = (NUM_TBUF * MP) < 32 ? 32 : NUM_TBUF * MP;
+  constexpr int COLS = MP / 2;                // token columns per promotion thread
+  constexpr int SFA_CHUNK = 32;               // K blocks of token scales staged at once
+  constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, MP);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);
+  __nv_bfloat16* s_c = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * STAGE_BYTES);  // [MP][128]
+  float* s_sfa = reinterpret_cast<float*>(s_c + MP * kBlockM);                          // [SFA_CHUNK][MP]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_sfa + SFA_CHUNK * MP);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + NUM_TBUF;
+  uint64_t* mma_done = tempty + NUM_TBUF;
+  uint64_t* pbar = mma_done + 1;  // promotion-group barrier
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int P = gridDim.x;
+  const int KB = p.num_kb;
+  const long long U = static_cast<long long>(p.n_tiles) * KB;
+  const long long u_begin = sk_begin(blockIdx.x, P, U);
+  const long long u_end = sk_begin(blockIdx.x + 1, P, U);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
+    mbar_init(mma_done, 1);
+    mbar_init(pbar, kPromoWarps * 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0) { prefetch_tmap(&tmW); prefetch_tmap(&tmT); }
+  if (warp == kMmaWarp) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();  // each weight byte is read once
+      const uint64_t pol_t = l2_policy_evict_last();   // tokens are re-read by every CTA
+      uint32_t stage = 0, phase = 0;
+      uint64_t issued = 0;
+      bool ok = true;
+      for (long long u = u_begin; u < u_end && ok;) {
+        const int t = static_cast<int>(u / KB);
+        const int kb0 = static_cast<int>(u - static_cast<long long>(t) * KB);
+        const long long tile_end = static_cast<long long>(t + 1) * KB;
+        const int kb1 = static_cast<int>((u_end < tile_end ? u_end : tile_end) - static_cast<long long>(t) * KB);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          uint8_t* sw = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_2d(sw, &tmW, &full[stage], kb * kBlockK, t * kBlockM, pol_w);
+          tma_load_2d(sw + W_BYTES, &tmT, &full[stage], kb * kBlockK, 0, pol_t);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        u = static_cast<long long>(t) * KB + kb1;
+      }
+      if (!ok) {
+        const uint64_t first = issued > STAGES ? issued - STAGES : 0;
+        for (uint64_t i = first; i < issued; ++i)
+          mbar_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
+      bool ok = true;
+      for (long long u = u_begin; u < u_end && ok;) {
+        const int t = static_cast<int>(u / KB);
+        const int kb0 = static_cast<int>(u - static_cast<long long>(t) * KB);
+        const long long tile_end = static_cast<long long>(t + 1) * KB;
+        const int kb1 = static_cast<int>((u_end < tile_end ? u_end : tile_end) - static_cast<long long>(t) * KB);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + tb * MP;
+          const uint32_t sw = smem_addr(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = smem_desc_k128_sw128(sw);
+          const uint64_t bdesc = smem_desc_k128_sw128(sw + W_BYTES);
+#pragma unroll
+          for (int j = 0; j < kBlockK / 32; ++j)
+            mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+          mma_commit(&empty[stage]);
+          mma_commit(&tfull[tb]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+        }
+        u = static_cast<long long>(t) * KB + kb1;
+      }
+      mma_commit(mma_done);
+      mbar_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------ promotion + fix-up + epilogue
+    const int q = warp & 3;
+    const int h = warp >> 2;
+    const int nl = q * 32 + lane;   // weight row within the n-tile (TMEM lane)
+    const int tid = threadIdx.x;    // 0..255 among promotion threads
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    uint32_t tb = 0, tphase = 0, pphase = 0;
+    bool ok = true;
+    bool first_segment = true;
+    for (long long u = u_begin; u < u_end && ok;) {
+      const int t = static_cast<int>(u / KB);
+      const int kb0 = static_cast<int>(u - static_cast<long long>(t) * KB);
+      const long long tile_end = static_cast<long long>(t + 1) * KB;
+      const int kb1 = static_cast<int>((u_end < tile_end ? u_end : tile_end) - static_cast<long long>(t) * KB);
+      const float* sb_ptr = p.sfb + static_cast<size_t>(t) * KB;
+
+      float acc[COLS];
+#pragma unroll
+      for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+
+      int chunk0 = -1;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (kb >= chunk0 + SFA_CHUNK || chunk0 < 0) {
+          // stage token scales sfa[kb..kb+SFA_CHUNK)[0..MP) (zero past M)
+          if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+          chunk0 = kb;
+          for (int i = tid; i < SFA_CHUNK * MP; i += kPromoWarps * 32) {
+            const int kk = chunk0 + i / MP, mm = i % MP;
+            s_sfa[i] = (kk < kb1 && mm < p.M) ? __ldg(p.sfa + static_cast<size_t>(kk) * p.ld + mm) : 0.0f;
+          }
+          if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        }
+        const float sb = __ldg(sb_ptr + kb);
+        if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + lane_off + tb * MP + h * COLS;
+        uint32_t v[COLS];
+        if constexpr (COLS == 16) {
+          uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+          tmem_ld_32x32b_x16(taddr, r16);
+        } else {
+#pragma unroll
+          for (int c0 = 0; c0 < COLS; c0 += 32) {
+            uint32_t (&r32)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + c0);
+            tmem_ld_32x32b_x32(taddr + c0, r32);
+          }
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[tb]);
+        const float4* sf4 = reinterpret_cast<const float4*>(s_sfa + (kb - chunk0) * MP + h * COLS);
+#pragma unroll
+        for (int j = 0; j < COLS; j += 4) {
+          const float4 a4 = sf4[j / 4];
+          acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), a4.x * sb, acc[j + 0]);
+          acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), a4.y * sb, acc[j + 1]);
+          acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), a4.z * sb, acc[j + 2]);
+          acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), a4.w * sb, acc[j + 3]);
+        }
+        if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+      }
+      if (!ok) break;
+
+      const bool whole = (kb0 == 0 && kb1 == KB);
+      bool do_store = whole;
+      if (!whole) {
+        // publish this CTA's partial, then let the last of the tile's CTAs sum them
+        const int slot = 2 * blockIdx.x + (first_segment ? 0 : 1);
+        float* wp = p.ws + static_cast<size_t>(slot) * MP * kBlockM + nl;
+#pragma unroll
+        for (int j = 0; j < COLS; ++j) wp[static_cast<size_t>(h * COLS + j) * kBlockM] = acc[j];
+        __threadfence();
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        const long long tu0 = static_cast<long long>(t) * KB;
+        const int c_first = sk_owner(tu0, P, U);
+        const int c_last = sk_owner(tu0 + KB - 1, P, U);
+        if (tid == 0) {
+          const int prev = atomicAdd(p.counters + t, 1);
+          const int last = (prev == c_last - c_first);
+          if (last) p.counters[t] = 0;  // ready for the next launch
+          *s_last = last;
+        }
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        if (*s_last) {
+          __threadfence();
+#pragma unroll
+          for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+          for (int c = c_first; c <= c_last; ++c) {
+            const int cs = 2 * c + (sk_begin(c, P, U) >= tu0 ? 0 : 1);
+            const float* rp = p.ws + static_cast<size_t>(cs) * MP * kBlockM + nl;
+#pragma unroll
+            for (int j = 0; j < COLS; ++j) acc[j] += __ldcg(rp + static_cast<size_t>(h * COLS + j) * kBlockM);
+          }
+          do_store = true;
+        }
+      }
+      if (do_store) {
+        // transpose through shared memory: s_c[m][nl], then 16-byte row stores of C[m, t*128 ..]
+#pragma unroll
+        for (int j = 0; j < COLS; ++j) s_c[(h * COLS + j) * kBlockM + nl] = __float2bfloat16_rn(acc[j]);
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        const int rows = p.M < MP ? p.M : MP;
+        const int n_base = t * kBlockM;
+        for (int i = tid; i < rows * (kBlockM / 8); i += kPromoWarps * 32) {
+          const int mm = i / (kBlockM / 8), ch = i % (kBlockM / 8);
+          if (n_base + ch * 8 < p.N) {
+            const uint4 v = *reinterpret_cast<const uint4*>(s_c + mm * kBlockM + ch * 8);
+            *reinterpret_cast<uint4*>(p.C + static_cast<size_t>(mm) * p.N + n_base + ch * 8) = v;
+          }
+        }
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+      }
+      first_segment = false;
+      u = static_cast<long long>(t) * KB + kb1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status);
+}
+
+}  // namespace fg

@@ -1,0 +1,359 @@
+// fp8gemm_api.cu -- host side of the C ABI declared in include/fp8gemm.h:
+// argument validation, TMA tensor-map encoding, kernel selection and launch.
+// Every GEMM call is one kernel launch on the caller's stream; nothing here
+// allocates after fg_init, reads device memory or synchronises.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fp8_gemm_kernels.cuh"
+#include "fp8gemm.h"
+
+namespace {
+
+using fg::kBlockK;
+using fg::kBlockM;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxSwapMP = 128;
+constexpr int kCounterCapacity = 1 << 16;  // n-tiles of 128 rows: N <= 8,388,608 on the stream-K path
+
+struct DeviceState {
+  bool ready = false;
+  int sms = 0;
+  int* status = nullptr;
+  float* ws = nullptr;
+  int* counters = nullptr;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+std::atomic<int> g_dense_path{0};
+std::atomic<uint64_t> g_launches{0};
+
+// tiled kernel configuration
+constexpr int kTiledBN = 128;
+constexpr int kTiledStages = 6;
+constexpr int kTiledTbuf = 4;
+
+template <int BN, int STAGES>
+constexpr size_t tiled_smem_bytes() {
+  return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBlockM + BN) * kBlockK + 256 /*barriers*/ +
+         4 * (fg::kMaskedMaxGroups + 1) /*masked prefix*/;
+}
+
+template <int MP>
+constexpr int swap_stages() {
+  return MP == 128 ? 5 : (MP == 64 ? 7 : 8);
+}
+
+template <int MP, int STAGES>
+constexpr size_t swap_smem_bytes() {
+  return 1024 + static_cast<size_t>(STAGES) * (kBlockM + MP) * kBlockK + MP * kBlockM * 2 /*C staging*/ +
+         32 * MP * 4 /*token scales*/ + 256 /*barriers*/;
+}
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+DeviceState* state_for_current(fg_status* err) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices || !g_dev[dev].ready) {
+    *err = FG_ERR_NOT_INITIALIZED;
+    return nullptr;
+  }
+  return &g_dev[dev];
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// 3-D map over e4m3 codes: dims {K, rows, groups}, box {128, box_rows, 1}, 128-byte swizzle,
+// out-of-bounds elements read as zero.
+bool encode_fp8_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t groups,
+                    uint32_t box_rows) {
+  cuuint64_t dims[3] = {K, rows, groups};
+  cuuint64_t strides[2] = {K, K * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockK), box_rows, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_fp8_map_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+  cuuint64_t dims[2] = {K, rows};
+  cuuint64_t strides[1] = {K};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockK), box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// One instantiation per kernel, so the once-per-device flag below is per kernel.
+template <auto KERNEL>
+fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap& m0, const CUtensorMap& m1,
+                 const void* params_ptr) {
+  // the opt-in shared-memory size is a per-function attribute: set once per device (so that a
+  // call made during stream capture issues no attribute change)
+  const auto kernel = KERNEL;
+  static std::atomic<uint64_t> configured{0};
+  const int dev = current_device();
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load(std::memory_order_acquire) & bit)) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+      return FG_ERR_CUDA;
+    configured.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  void* args[3] = {const_cast<CUtensorMap*>(&m0), const_cast<CUtensorMap*>(&m1), const_cast<void*>(params_ptr)};
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(fg::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(kernel), args);
+  if (e != cudaSuccess) return FG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FG_OK;
+}
+
+// common argument checks for the FP8 operands
+fg_status check_common(const void* A, const float* sfa, const void* B, const float* sfb, const void* C, int N,
+                       int K) {
+  if (!A || !sfa || !B || !sfb || !C) return FG_ERR_INVALID_ARG;
+  if (N < 0 || K <= 0) return FG_ERR_INVALID_ARG;
+  if (K % 16 != 0 || N % 8 != 0) return FG_ERR_ALIGNMENT;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sfa, 4) || !aligned(sfb, 4))
+    return FG_ERR_ALIGNMENT;
+  return FG_OK;
+}
+
+template <int MODE>
+fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                    const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream) {
+  constexpr int BN = kTiledBN;
+  constexpr int STAGES = kTiledStages;
+  fg::TiledParams p;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.m_indices = m_indices;
+  p.masked_m = masked_m;
+  p.status = st->status;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.G = G;
+  p.ld = fg_sfa_ld(M);
+  p.num_kb = (K + kBlockK - 1) / kBlockK;
+  p.num_nb = (N + kBlockK - 1) / kBlockK;
+  p.m_blocks = (M + kBlockM - 1) / kBlockM;
+  p.n_blocks = (N + BN - 1) / BN;
+
+  CUtensorMap mA, mB;
+  const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;
+  const uint64_t groupsB = (MODE == fg::kDense) ? 1 : static_cast<uint64_t>(G);
+  if (!encode_fp8_map(&mA, A, K, M, groupsA, kBlockM)) return FG_ERR_CUDA;
+  if (!encode_fp8_map(&mB, B, K, N, groupsB, BN)) return FG_ERR_CUDA;
+
+  long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
+  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, kTiledTbuf, MODE>>(
+      dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, mA, mB, &p);
+}
+
+template <int MP>
+fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                   int M, int N, int K, cudaStream_t stream) {
+  constexpr int STAGES = swap_stages<MP>();
+  fg::SwapParams p;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.ws = st->ws;
+  p.counters = st->counters;
+  p.status = st->status;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ld = fg_sfa_ld(M);
+  p.num_kb = (K + kBlockK - 1) / kBlockK;
+  p.n_tiles = (N + kBlockM - 1) / kBlockM;
+  if (p.n_tiles > kCounterCapacity) return FG_ERR_UNSUPPORTED;
+
+  CUtensorMap mW, mT;
+  if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
+  if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
+  const long long units = static_cast<long long>(p.n_tiles) * p.num_kb;
+  const int grid = static_cast<int>(units < st->sms ? units : st->sms);
+  return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(grid), swap_smem_bytes<MP, STAGES>(), stream,
+                                                               mW, mT, &p);
+}
+
+}  // namespace
+
+extern "C" {
+
+fg_status fg_init(int device) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (device < 0 || device >= kMaxDevices) return FG_ERR_INVALID_ARG;
+  if (cudaSetDevice(device) != cudaSuccess) return FG_ERR_CUDA;
+  DeviceState& st = g_dev[device];
+  if (st.ready) return FG_OK;
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return FG_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device) != cudaSuccess)
+    return FG_ERR_CUDA;
+  if (major != 10 || minor != 0) return FG_ERR_UNSUPPORTED;  // built for sm_100a only
+  if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return FG_ERR_CUDA;
+  const size_t ws_floats = static_cast<size_t>(2) * st.sms * kMaxSwapMP * kBlockM;
+  if (cudaMalloc(&st.status, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+  if (cudaMalloc(&st.ws, ws_floats * sizeof(float)) != cudaSuccess) return FG_ERR_CUDA;
+  if (cudaMalloc(&st.counters, kCounterCapacity * sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+  if (cudaMemset(st.status, 0, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+  if (cudaMemset(st.counters, 0, kCounterCapacity * sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FG_ERR_CUDA;
+  st.ready = true;
+  return FG_OK;
+}
+
+void fg_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  int prev = -1;
+  cudaGetDevice(&prev);
+  for (int d = 0; d < kMaxDevices; ++d) {
+    DeviceState& st = g_dev[d];
+    if (!st.ready) continue;
+    cudaSetDevice(d);
+    cudaFree(st.status);
+    cudaFree(st.ws);
+    cudaFree(st.counters);
+    st = DeviceState();
+  }
+  if (prev >= 0) cudaSetDevice(prev);
+}
+
+int fg_m_alignment(void) { return kBlockM; }
+
+int fg_sfa_ld(int M) { return M <= 0 ? 0 : (M + 3) / 4 * 4; }
+
+int fg_set_dense_path(int path) {
+  if (path < 0 || path > 2) return g_dense_path.load();
+  return g_dense_path.exchange(path);
+}
+
+uint64_t fg_launch_count(void) { return g_launches.load(); }
+
+fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
+                      int K, void* stream) {
+  if (M < 0 || N < 0) return FG_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FG_OK;
+  fg_status s = check_common(A, sfa, B, sfb, C, N, K);
+  if (s != FG_OK) return s;
+  if (static_cast<long long>(M) * K >= (1ll << 40) || static_cast<long long>(N) * K >= (1ll << 40))
+    return FG_ERR_UNSUPPORTED;
+  DeviceState* st = state_for_current(&s);
+  if (!st) return s;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int path = g_dense_path.load();
+  const bool swap = (path == 2) || (path == 0 && M <= kMaxSwapMP);
+  if (swap) {
+    if (M > kMaxSwapMP) return FG_ERR_UNSUPPORTED;
+    if (M <= 32) return run_swap<32>(st, A, sfa, B, sfb, C, M, N, K, cs);
+    if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs);
+    return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs);
+  }
+  return run_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs);
+}
+
+fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                                      const int* m_indices, int M_total, int G, int N, int K, void* stream) {
+  if (M_total < 0 || N < 0 || G < 0) return FG_ERR_INVALID_ARG;
+  if (M_total == 0 || N == 0) return FG_OK;
+  if (G == 0) return FG_ERR_INVALID_ARG;
+  fg_status s = check_common(A, sfa, B, sfb, C, N, K);
+  if (s != FG_OK) return s;
+  if (!m_indices) return FG_ERR_INVALID_ARG;
+  if (!aligned(m_indices, 4)) return FG_ERR_ALIGNMENT;
+  if (static_cast<long long>(M_total) * K >= (1ll << 40) || static_cast<long long>(G) * N * K >= (1ll << 40))
+    return FG_ERR_UNSUPPORTED;
+  DeviceState* st = state_for_current(&s);
+  if (!st) return s;
+  return run_tiled<fg::kContiguous>(st, A, sfa, B, sfb, C, m_indices, nullptr, M_total, G, N, K,
+                                    static_cast<cudaStream_t>(stream));
+}
+
+fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                                  const int* masked_m, int G, int Mmax, int N, int K, void* stream) {
+  if (G < 0 || Mmax < 0 || N < 0) return FG_ERR_INVALID_ARG;
+  if (G == 0 || Mmax == 0 || N == 0) return FG_OK;
+  fg_status s = check_common(A, sfa, B, sfb, C, N, K);
+  if (s != FG_OK) return s;
+  if (!masked_m) return FG_ERR_INVALID_ARG;
+  if (!aligned(masked_m, 4)) return FG_ERR_ALIGNMENT;
+  if (G > fg::kMaskedMaxGroups) return FG_ERR_UNSUPPORTED;
+  if (static_cast<long long>(G) * Mmax * K >= (1ll << 40) || static_cast<long long>(G) * N * K >= (1ll << 40))
+    return FG_ERR_UNSUPPORTED;
+  DeviceState* st = state_for_current(&s);
+  if (!st) return s;
+  return run_tiled<fg::kMasked>(st, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
+                                static_cast<cudaStream_t>(stream));
+}
+
+fg_status fg_get_device_status(void* stream) {
+  fg_status s;
+  DeviceState* st = state_for_current(&s);
+  if (!st) return s;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FG_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FG_ERR_CUDA;
+  if (v != 0) {
+    // a kernel gave up early: clear the word and the stream-K counters it may have left behind
+    if (cudaMemset(st->status, 0, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+    if (cudaMemset(st->counters, 0, kCounterCapacity * sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return FG_ERR_CUDA;
+    return static_cast<fg_status>(v);
+  }
+  return FG_OK;
+}
+
+const char* fg_status_string(fg_status status) {
+  switch (status) {
+    case FG_OK: return "FG_OK";
+    case FG_ERR_INVALID_ARG: return "FG_ERR_INVALID_ARG";
+    case FG_ERR_ALIGNMENT: return "FG_ERR_ALIGNMENT";
+    case FG_ERR_UNSUPPORTED: return "FG_ERR_UNSUPPORTED";
+    case FG_ERR_NOT_INITIALIZED: return "FG_ERR_NOT_INITIALIZED";
+    case FG_ERR_CUDA: return "FG_ERR_CUDA";
+    case FG_ERR_TIMEOUT: return "FG_ERR_TIMEOUT";
+  }
+  return "FG_ERR_UNKNOWN";
+}
+
+}  // extern "C"

@@ -1,0 +1,79 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before touching the GPU."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import moe_grouped_gemm_08_b200 as fg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8gemm.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\(", text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while")))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("fp8_gemm_nt", "fp8_gemm_grouped_contiguous", "fp8_gemm_grouped_masked", "fg_init",
+                     "fg_m_alignment", "fg_sfa_ld", "fg_get_device_status", "fg_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(str(fg.LIB_PATH))
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in fp8gemm.h but not exported"
+
+
+def test_queries():
+    assert fg.get_m_alignment_for_contiguous_layout() == 128
+    assert [fg.sfa_ld(m) for m in (0, 1, 4, 5, 128, 1025)] == [0, 4, 4, 8, 128, 1028]
+    assert fg.STATUS_NAMES[6] == "FG_ERR_TIMEOUT"
+    assert fg.lib.fg_status_string(99) == b"FG_ERR_UNKNOWN"
+
+
+def test_dense_path_switch():
+    old = fg.set_dense_path(1)
+    assert fg.set_dense_path(2) == 1
+    assert fg.set_dense_path(7) == 2  # ignored
+    fg.set_dense_path(old)
+
+
+NULL = None
+P16 = 0x10000  # a fake 16-byte-aligned address: these calls must fail before any dereference
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((NULL, P16, P16, P16, P16, 64, 128, 128, NULL), 1),     # null A
+    ((P16, P16, P16, P16, P16, 64, 128, 0, NULL), 1),        # K = 0
+    ((P16, P16, P16, P16, P16, -1, 128, 128, NULL), 1),      # negative M
+    ((P16, P16, P16, P16, P16, 64, 128, 120, NULL), 2),      # K % 16
+    ((P16, P16, P16, P16, P16, 64, 100, 128, NULL), 2),      # N % 8
+    ((P16 + 8, P16, P16, P16, P16, 64, 128, 128, NULL), 2),  # A misaligned
+    ((P16, P16 + 2, P16, P16, P16, 64, 128, 128, NULL), 2),  # sfa misaligned
+    ((P16, P16, P16, P16, P16, 0, 128, 128, NULL), 0),       # M = 0: no-op
+    ((NULL, NULL, NULL, NULL, NULL, 0, 0, 0, NULL), 0),      # empty: no-op
+])
+def test_dense_argument_errors(args, expect):
+    assert fg.lib.fp8_gemm_nt(*args) == expect
+
+
+def test_grouped_argument_errors():
+    L = fg.lib
+    assert L.fp8_gemm_grouped_contiguous(P16, P16, P16, P16, P16, NULL, 256, 2, 128, 128, NULL) == 1
+    assert L.fp8_gemm_grouped_contiguous(P16, P16, P16, P16, P16, P16, 256, 0, 128, 128, NULL) == 1
+    assert L.fp8_gemm_grouped_contiguous(P16, P16, P16, P16, P16, P16 + 2, 256, 2, 128, 128, NULL) == 2
+    assert L.fp8_gemm_grouped_contiguous(P16, P16, P16, P16, P16, P16, 0, 2, 128, 128, NULL) == 0
+    assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, NULL, 2, 64, 128, 128, NULL) == 1
+    assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, P16, 2000, 64, 128, 128, NULL) == 3
+    assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, P16, 2, 64, 128, 136, NULL) == 2
+    assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, P16, 0, 64, 128, 128, NULL) == 0

@@ -1,0 +1,218 @@
+"""GPU parity: the CUDA path (through the C ABI binding) against the CPU oracle.
+
+Every comparison uses the stated tolerance (tests/gpu_helpers.py):
+elementwise |c - r| <= 0.01 |r| + 1e-3 max|r| and per matrix
+1 - 2 sum(c r) / sum(c^2 + r^2) < 1e-5.  Full-size workloads are checked in full
+where the oracle finishes in seconds (decode sweep, masked), otherwise on sampled
+rows (prefill, contiguous), in the launch configuration the benchmark times.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from synth import workloads
+from tests.gpu_helpers import bits_of, close, dense_dev, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fg():
+    import moe_grouped_gemm_08_b200 as lib
+    torch.cuda.set_device(0)
+    lib.init(0)
+    yield lib
+    lib.set_dense_path(0)
+
+
+def canary_like(shape):
+    """bf16 tensor whose every element has the bit pattern 0xFFFF (a NaN nobody writes)."""
+    return torch.full(shape, -1, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+
+
+def run_dense(fg, case, path):
+    old = fg.set_dense_path(path)
+    try:
+        A, sfa, B, sfb = dense_dev(case)
+        C = fg.gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb)
+        torch.cuda.synchronize()
+    finally:
+        fg.set_dense_path(old)
+    return bits_of(C)
+
+
+def sample_rows(M, n, seed):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, M // 2, M - 129, M - 128, M - 1]
+    rows = np.unique(np.concatenate([[r for r in fixed if 0 <= r < M], rng.integers(0, M, n)]))
+    return rows.astype(np.int32)
+
+
+# --------------------------------------------------------------------------- dense
+@pytest.mark.parametrize("path", [1, 2])
+def test_dense_single(fg, path):
+    w = workloads.dense_single()[0]
+    case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"])
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
+    close(run_dense(fg, case, path), ref, f"dense_single path={path}")
+
+
+ODD = [(1, 8, 16), (7, 136, 272), (33, 4104, 2048), (64, 264, 640), (100, 2112, 384), (128, 1000, 256),
+       (129, 520, 256), (200, 136, 1152), (300, 392, 128), (513, 2048, 3072)]
+
+
+@pytest.mark.parametrize("M,N,K", ODD)
+def test_dense_odd_shapes(fg, M, N, K):
+    case = synth.dense_case(100 + M, M, N, K, row_scaled=True)
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
+    for path in ([1, 2] if M <= 128 else [1]):
+        close(run_dense(fg, case, path), ref, f"odd {M}x{N}x{K} path={path}")
+
+
+@pytest.mark.parametrize("w", workloads.decode_sweep(), ids=lambda w: w["name"])
+def test_decode_sweep_full(fg, w):
+    case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"], row_scaled=True)
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
+    close(run_dense(fg, case, 0), ref, w["name"])
+    if w["N"] * w["K"] <= 7168 * 7168:
+        close(run_dense(fg, case, 1), ref, w["name"] + " tiled")
+
+
+@pytest.mark.parametrize("w", workloads.prefill(), ids=lambda w: w["name"])
+def test_prefill_sampled_rows(fg, w):
+    case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"])
+    rows = sample_rows(w["M"], 40, w["seed"])
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"], rows=rows)
+    got = run_dense(fg, case, 0)
+    close(got[rows], ref, w["name"])
+
+
+def test_stream_k_deterministic(fg):
+    w = workloads.decode_sweep()[0]
+    case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"], row_scaled=True)
+    a = run_dense(fg, case, 2)
+    b = run_dense(fg, case, 2)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_dense_m_zero_is_noop(fg):
+    A = torch.zeros((0, 128), dtype=torch.uint8, device="cuda")
+    sfa = torch.zeros((1, 0), dtype=torch.float32, device="cuda")
+    B = torch.zeros((128, 128), dtype=torch.uint8, device="cuda")
+    sfb = torch.ones((1, 1), dtype=torch.float32, device="cuda")
+    C = fg.gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb)
+    assert C.shape == (0, 128)
+
+
+# --------------------------------------------------------------------------- contiguous
+def run_contig(fg, case, C=None):
+    A, sfa = to_dev(case["A"]), to_dev(case["sfa"])
+    B, sfb = to_dev(case["B"]), to_dev(case["sfb"])
+    mi = to_dev(case["m_indices"])
+    if C is None:
+        C = canary_like((case["M"], case["N"]))
+    fg.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, mi, C=C)
+    torch.cuda.synchronize()
+    return bits_of(C)
+
+
+def test_contiguous_odd_padding(fg):
+    case = synth.contiguous_case(41, [100, 0, 300, 37, 128, 1], N=264, K=384)
+    got = run_contig(fg, case)
+    canary = np.full((case["M"], case["N"]), 0xFFFF, dtype=np.uint16)
+    ref = oracle.grouped_contiguous(case["A"], case["sfa"], case["B"], case["sfb"], case["m_indices"], C=canary)
+    live = case["m_indices"] >= 0
+    close(got[live], ref[live], "contiguous odd")
+    assert np.all(got[~live] == 0xFFFF), "padding rows were written"
+
+
+def test_contiguous_out_of_range_index_is_skipped(fg):
+    case = synth.contiguous_case(42, [128, 128, 128], N=136, K=256)
+    mi = case["m_indices"].copy()
+    mi[256:384] = 7  # >= G: treated as padding
+    case["m_indices"] = mi
+    got = run_contig(fg, case)
+    assert np.all(got[256:] == 0xFFFF)
+    ref = oracle.grouped_contiguous(case["A"], case["sfa"], case["B"], case["sfb"], mi)
+    close(got[:256], ref[:256], "contiguous index >= G")
+
+
+@pytest.mark.parametrize("w", workloads.contiguous(), ids=lambda w: w["name"])
+def test_contiguous_full_size_sampled(fg, w):
+    case = synth.contiguous_case(w["seed"], [w["M_per_group"]] * w["G"], w["N"], w["K"])
+    got = run_contig(fg, case, C=torch.empty((case["M"], case["N"]), dtype=torch.bfloat16, device="cuda"))
+    rows = sample_rows(case["M"], 48, w["seed"])
+    ref = oracle.grouped_contiguous(case["A"], case["sfa"], case["B"], case["sfb"], case["m_indices"], rows=rows)
+    close(got[rows], ref, w["name"])
+
+
+# --------------------------------------------------------------------------- masked
+def masked_dev(case):
+    return (to_dev(case["A"]), to_dev(case["sfa"]), to_dev(case["B"]), to_dev(case["sfb"]),
+            to_dev(case["masked_m"]))
+
+
+def check_masked(got, case, what):
+    G, Mmax, N = case["G"], case["Mmax"], case["N"]
+    canary = np.full((G, Mmax, N), 0xFFFF, dtype=np.uint16)
+    ref = oracle.grouped_masked(case["A"], case["sfa"], case["B"], case["sfb"], case["masked_m"], C=canary)
+    for g in range(G):
+        v = min(int(case["masked_m"][g]), Mmax)
+        if v:
+            close(got[g, :v], ref[g, :v], f"{what} g={g}")
+        assert np.all(got[g, v:] == 0xFFFF), f"{what}: rows past masked_m[{g}]={v} were written"
+
+
+@pytest.mark.parametrize("w", workloads.masked(), ids=lambda w: w["name"])
+def test_masked_under_cuda_graph(fg, w):
+    case = synth.masked_case(w["seed"], w["G"], w["Mmax"], w["N"], w["K"])
+    A, sfa, B, sfb, mm = masked_dev(case)
+    C = canary_like((w["G"], w["Mmax"], w["N"]))
+    fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, mm, C=C)  # warm-up outside capture
+    C.view(torch.int16).fill_(-1)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, mm, C=C)
+    C.view(torch.int16).fill_(-1)
+    graph.replay()
+    torch.cuda.synchronize()
+    check_masked(bits_of(C), case, w["name"])
+    # new counts written into the same device buffer, same graph replayed
+    if w["G"] >= 2:
+        new = np.array(case["masked_m"][::-1], dtype=np.int32)
+        mm.copy_(torch.from_numpy(new).cuda())
+        C.view(torch.int16).fill_(-1)
+        graph.replay()
+        torch.cuda.synchronize()
+        case2 = dict(case, masked_m=new)
+        check_masked(bits_of(C), case2, w["name"] + " replay")
+    else:
+        for cnt in (0, 333):
+            mm.fill_(cnt)
+            C.view(torch.int16).fill_(-1)
+            graph.replay()
+            torch.cuda.synchronize()
+            check_masked(bits_of(C), dict(case, masked_m=np.array([cnt], np.int32)), f"{w['name']} m={cnt}")
+    del graph
+
+
+def test_masked_counts_edge_cases(fg):
+    case = synth.masked_case(51, 3, 200, 136, 256, masked_m=[0, 0, 0])
+    A, sfa, B, sfb, mm = masked_dev(case)
+    C = canary_like((3, 200, 136))
+    fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, mm, C=C)
+    torch.cuda.synchronize()
+    assert np.all(bits_of(C) == 0xFFFF)
+    mm.copy_(torch.tensor([500, 1, 129], dtype=torch.int32, device="cuda"))  # 500 > Mmax: clamped
+    fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, mm, C=C)
+    torch.cuda.synchronize()
+    check_masked(bits_of(C), dict(case, masked_m=np.array([200, 1, 129], np.int32)), "masked edge")
+
+
+def test_device_status_clean(fg):
+    assert fg.device_status() == 0
