@@ -1,0 +1,536 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 block-scaled NT GEMM on B200.
+
+One step = one pass of the chosen workload (default: the dense decode sweep, M in
+{64,128} x six (N,K) DeepSeek-V3/R1 shapes = 12 GEMM launches) over inputs
+already resident in HBM.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Timing: each step is replayed from a CUDA graph (the masked-layout call is made
+for graphs; the dense calls are captured the same way so that host launch cost
+does not hide in the device timeline).  Inputs rotate over R copies whose total
+size is several times the 126 MB L2, so every launch reads its operands from HBM.
+The timed region is bracketed by a barrier and torch.cuda.synchronize() on both
+sides and measured with CUDA events on the launching stream; multi-GPU runs take
+the max over ranks (independent replicas: the GEMM needs no exchange step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+from synth import workloads  # noqa: E402
+
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
+KERNEL_SOURCES = ["moe_grouped_gemm_08_b200/csrc/fp8_gemm_kernels.cuh",
+                  "moe_grouped_gemm_08_b200/csrc/sm100_ptx.cuh",
+                  "moe_grouped_gemm_08_b200/csrc/fp8gemm_api.cu"]
+
+
+# ---------------------------------------------------------------------------- helpers
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained") if k in d}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel: str, workload: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    entry = d.get(f"{kernel}:{workload}")
+    if not entry or entry.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return entry
+
+
+def cdiv(a, b):
+    return (a + b - 1) // b
+
+
+def workload_list(name: str):
+    table = {"decode_sweep": workloads.decode_sweep, "dense_single": workloads.dense_single,
+             "prefill": workloads.prefill, "contiguous": workloads.contiguous, "masked": workloads.masked}
+    if name not in table:
+        raise SystemExit(f"unknown workload {name}; choose from {sorted(table)}")
+    return name, table[name]()
+
+
+def make_case(w):
+    if "Mmax" in w:
+        return synth.masked_case(w["seed"], w["G"], w["Mmax"], w["N"], w["K"])
+    if "M_per_group" in w:
+        return synth.contiguous_case(w["seed"], [w["M_per_group"]] * w["G"], w["N"], w["K"])
+    return synth.dense_case(w["seed"], w["M"], w["N"], w["K"], row_scaled=w.get("row_scaled", False))
+
+
+def work_of(case):
+    """(flops, algorithmic bytes incl. scales, pages-style bytes A+B+C) of one call, valid rows only."""
+    N, K = case["N"], case["K"]
+    KB, NB = cdiv(K, 128), cdiv(N, 128)
+    if case["kind"] == "masked":
+        valid = np.minimum(case["masked_m"], case["Mmax"]).astype(np.int64)
+        Mv = int(valid.sum())
+        groups_used = int((valid > 0).sum())
+        G = case["G"]
+        flops = 2 * Mv * N * K
+        byt = Mv * K + groups_used * N * K + 2 * Mv * N + 4 * Mv * KB + 4 * groups_used * NB * KB
+        pages = G * case["Mmax"] * K + G * N * K + 2 * G * case["Mmax"] * N
+        return flops, byt, pages
+    if case["kind"] == "contiguous":
+        Mv = int((case["m_indices"] >= 0).sum())
+        G = case["G"]
+        flops = 2 * Mv * N * K
+        byt = Mv * K + G * N * K + 2 * Mv * N + 4 * Mv * KB + 4 * G * NB * KB
+        return flops, byt, Mv * K + G * N * K + 2 * Mv * N
+    M = case["M"]
+    flops = 2 * M * N * K
+    byt = M * K + N * K + 2 * M * N + 4 * M * KB + 4 * NB * KB
+    return flops, byt, M * K + N * K + 2 * M * N
+
+
+def kernel_name(case) -> str:
+    if case["kind"] == "dense" and case["M"] <= 128:
+        return "fp8_gemm_swap_streamk_kernel"
+    return "fp8_gemm_tiled_kernel"
+
+
+def upload(case, dev):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)  # noqa: E731
+    d = dict(A=t(case["A"]), sfa=t(case["sfa"]), B=t(case["B"]), sfb=t(case["sfb"]))
+    if case["kind"] == "masked":
+        d["masked_m"] = t(case["masked_m"])
+        d["C"] = torch.empty((case["G"], case["Mmax"], case["N"]), dtype=torch.bfloat16, device=dev)
+    elif case["kind"] == "contiguous":
+        d["m_indices"] = t(case["m_indices"])
+        d["C"] = torch.empty((case["M"], case["N"]), dtype=torch.bfloat16, device=dev)
+    else:
+        d["C"] = torch.empty((case["M"], case["N"]), dtype=torch.bfloat16, device=dev)
+    return d
+
+
+def call(fg, case, d, stream=None):
+    if case["kind"] == "masked":
+        return fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(d["A"], d["sfa"], d["B"], d["sfb"], d["masked_m"],
+                                                        C=d["C"], stream=stream)
+    if case["kind"] == "contiguous":
+        return fg.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(d["A"], d["sfa"], d["B"], d["sfb"], d["m_indices"],
+                                                            C=d["C"], stream=stream)
+    return fg.gemm_fp8_fp8_bf16_nt(d["A"], d["sfa"], d["B"], d["sfb"], C=d["C"], stream=stream)
+
+
+_CUDART = None
+
+
+def record_event_node(ev: torch.cuda.Event, stream: torch.cuda.Stream) -> None:
+    """Record `ev` on `stream` so that, during stream capture, it becomes an event-record node of the
+    graph (cudaEventRecordExternal): its timestamp is then readable after every replay."""
+    global _CUDART
+    import ctypes
+    if _CUDART is None:
+        _CUDART = ctypes.CDLL("libcudart.so.12")
+        _CUDART.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        _CUDART.cudaEventRecordWithFlags.restype = ctypes.c_int
+    rc = _CUDART.cudaEventRecordWithFlags(ctypes.c_void_p(ev.cuda_event), ctypes.c_void_p(stream.cuda_stream), 1)
+    if rc != 0:
+        raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms in the background."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        inside = [s for (ts, s) in self.samples if t0 - 0.05 <= ts <= t1 + 0.15]
+        note = None
+        if not inside:  # timed region shorter than the sampling period: nearest samples
+            inside = [min(self.samples, key=lambda x: abs(x[0] - (t0 + t1) / 2))[1]]
+            note = "timed region shorter than the 100 ms sampling period; nearest sample"
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(s[2]) for s in inside if num(s[2]) is not None]
+        smax = [num(s[3]) for s in inside if num(s[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in inside for i in range(4) if len(s) > 6 + i and s[6 + i] == "Active"})
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+               "reasons": reasons, "samples": len(inside)}
+        if note:
+            out["note"] = note
+        return out
+
+
+# ---------------------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if (args.impl == "ours" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world, local
+
+
+def barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[local])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------- CPU oracle timing
+def time_oracle(cases, row_fraction: float = 1.0):
+    """Time the CPU oracle as it stands over (a row sample of) the cases; returns (seconds, flops, desc)."""
+    import oracle  # the oracle is test infrastructure; only this leg of the benchmark runs it
+    flops = 0
+    t0 = time.perf_counter()
+    for c in cases:
+        if c["kind"] == "dense":
+            M = c["M"]
+            n = max(1, int(round(M * row_fraction)))
+            rows = np.linspace(0, M - 1, n).astype(np.int32)
+            oracle.gemm_nt(c["A"], c["sfa"], c["B"], c["sfb"], rows=rows if n < M else None)
+            flops += 2 * n * c["N"] * c["K"]
+        elif c["kind"] == "contiguous":
+            M = c["M"]
+            n = max(1, int(round(M * row_fraction)))
+            rows = np.linspace(0, M - 1, n).astype(np.int32)
+            oracle.grouped_contiguous(c["A"], c["sfa"], c["B"], c["sfb"], c["m_indices"], rows=rows)
+            flops += 2 * int((c["m_indices"][rows] >= 0).sum()) * c["N"] * c["K"]
+        else:
+            mm = np.minimum(c["masked_m"], c["Mmax"])
+            sub = np.maximum(1, np.round(mm * row_fraction)).astype(np.int32) * (mm > 0)
+            oracle.grouped_masked(c["A"], c["sfa"], c["B"], c["sfb"], sub)
+            flops += 2 * int(sub.sum()) * c["N"] * c["K"]
+    return time.perf_counter() - t0, flops, oracle.num_threads()
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on the same workload, rank 0 only."""
+    if rank != 0:
+        return
+    name, wl = workload_list(args.workload)
+    cases = [make_case(w) for w in wl]
+    full_flops = sum(work_of(c)[0] for c in cases)
+    # size each step so that warm-up + timed steps stay within about two minutes
+    probe_s, probe_flops, cores = time_oracle(cases, row_fraction=min(1.0, 0.05))
+    rate = probe_flops / max(probe_s, 1e-9)
+    budget_per_step = 120.0 / max(1, args.steps + args.warmup)
+    frac = float(min(1.0, max(1e-4, budget_per_step * rate / full_flops)))
+    for _ in range(args.warmup):
+        time_oracle(cases, frac)
+    total_s, total_flops = 0.0, 0
+    for _ in range(args.steps):
+        s, f, cores = time_oracle(cases, frac)
+        total_s += s
+        total_flops += f
+    value = total_flops / total_s / 1e12
+    sample = f"{frac:.4g} of the rows of every GEMM of the {name} workload per step (evenly spaced rows)"
+    line = {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "shapes": [w["name"] for w in wl]}, "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "FP8 TFLOPS & HBM GB/s per GEMM shape on 1xB200; % of FP8/HBM roofline"
+
+
+# ---------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local):
+    import moe_grouped_gemm_08_b200 as fg
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fg.init(local)
+    name, wl = workload_list(args.workload)
+    cases = [make_case(w) for w in wl]
+    works = [work_of(c) for c in cases]
+    step_flops = sum(w[0] for w in works)
+    step_bytes = sum(w[1] for w in works)
+    step_in_bytes = sum(c["A"].nbytes + c["B"].nbytes + c["sfa"].nbytes + c["sfb"].nbytes for c in cases)
+
+    # rotation: enough input copies that one copy is re-read only after > 3x L2 of other traffic
+    rot = max(2, min(8, cdiv(3 * L2_BYTES, max(1, step_in_bytes)) + 1))
+    devs = [[upload(c, dev) for c in cases] for _ in range(rot)]
+    stream = torch.cuda.Stream(device=dev)
+
+    # eager warm-up call per case (sets kernel attributes before capture), then capture one graph per copy
+    with torch.cuda.stream(stream):
+        for c, d in zip(cases, devs[0]):
+            call(fg, c, d, stream=stream)
+    stream.synchronize()
+    launches_before = fg.launch_count()
+    graphs = []       # kernels only: the timed region (consecutive launches may overlap via PDL)
+    for r in range(rot):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c, d in zip(cases, devs[r]):
+                call(fg, c, d, stream=stream)
+        graphs.append(g)
+    launches_per_step = (fg.launch_count() - launches_before) // rot
+    egraphs, gevents = [], []  # the same step with an event node around every launch: per-shape times
+    for r in range(rot):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(cases) + 1)]
+        for ev in evs:  # create the CUDA events outside capture
+            ev.record(stream)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i, (c, d) in enumerate(zip(cases, devs[r])):
+                record_event_node(evs[i], stream)
+                call(fg, c, d, stream=stream)
+            record_event_node(evs[-1], stream)
+        egraphs.append(g)
+        gevents.append(evs)
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    for k in range(args.warmup):
+        graphs[k % rot].replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    start.record(stream)
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            graphs[(args.warmup + k) % rot].replay()
+    end.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    barrier(world, local)
+    time.sleep(0.25)
+    clocks.stop()
+    elapsed_ms = start.elapsed_time(end)
+    elapsed_ms = max_over_ranks(elapsed_ms, world)
+    # per-shape device durations: a separate pass over the event-instrumented graphs
+    per_case_ms = [[] for _ in cases]
+    with torch.cuda.stream(stream):
+        for k in range(3 * rot):
+            egraphs[k % rot].replay()
+            stream.synchronize()
+            evs = gevents[k % rot]
+            for i in range(len(cases)):
+                per_case_ms[i].append(evs[i].elapsed_time(evs[i + 1]))
+    status = fg.device_status(stream)
+
+    total_flops = step_flops * args.steps * world
+    value = total_flops / (elapsed_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    shapes = []
+    sum_bytes_swap, sum_ms_swap, sum_ms_all = 0.0, 0.0, 0.0
+    for c, w, wk, ts in zip(cases, wl, works, per_case_ms):
+        ms = statistics.mean(ts)
+        tfl = wk[0] / (ms * 1e-3) / 1e12
+        gbs = wk[1] / (ms * 1e-3) / 1e9
+        t_roof = max(wk[0] / (fp8_peak * 1e12), wk[1] / (peaks["hbm_gbs"] * 1e9))
+        shapes.append({"name": w["name"], "us": round(ms * 1e3, 2), "tflops": round(tfl, 1), "gbs": round(gbs, 1),
+                       "pages_gbs": round(wk[2] / (ms * 1e-3) / 1e9, 1),
+                       "bound": "hbm" if wk[1] / (peaks["hbm_gbs"] * 1e9) > wk[0] / (fp8_peak * 1e12) else "tensor",
+                       "roofline_frac": round(t_roof / (ms * 1e-3), 3), "kernel": kernel_name(c)})
+        sum_ms_all += ms
+        if kernel_name(c) == kernel_name(cases[0]):
+            sum_bytes_swap += wk[1]
+            sum_ms_swap += ms
+    dom = kernel_name(cases[0])
+    dom_bound = "hbm" if all(s["bound"] == "hbm" for s in shapes if s["kernel"] == dom) else "tensor"
+    single_kernel = all(kernel_name(c) == dom for c in cases)
+    if single_kernel:
+        # every launch of the timed region is this kernel: its average launch duration is the
+        # timed region divided by the launches (inter-kernel gaps included)
+        sum_ms_swap = elapsed_ms / args.steps
+        sum_ms_all = sum_ms_swap
+    if dom_bound == "hbm":
+        achieved = sum_bytes_swap / (sum_ms_swap * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4)}
+    else:
+        dom_flops = sum(wk[0] for c, wk in zip(cases, works) if kernel_name(c) == dom)
+        achieved = dom_flops / (sum_ms_swap * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
+                "frac": round(achieved / fp8_peak, 4)}
+    tr = load_traffic(dom, name)
+    roof["traffic"] = tr["dram_bytes_per_launch"] if tr else None
+    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if dom_bound == 'hbm' else 'bf16_tflops x 2 nominal fp8/bf16'})"
+    roof["kernel"] = dom
+    roof["launch_share"] = round(sum_ms_swap / sum_ms_all, 4) if sum_ms_all else None
+    roof["bytes_per_launch_def"] = "A + B + C + fp32 scales, valid rows, per launch; summed over the step"
+    roof["timing"] = ("timed region / launches" if single_kernel else
+                      "event-instrumented pass after the timed region")
+
+    # end to end through the public API with host buffers: H2D of the step's inputs, GEMMs, D2H of C
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    host = []
+    for c in cases:
+        h = {k: torch.from_numpy(np.ascontiguousarray(c[k])).pin_memory() for k in ("A", "sfa", "B", "sfb")}
+        if c["kind"] == "masked":
+            h["masked_m"] = torch.from_numpy(c["masked_m"]).pin_memory()
+        if c["kind"] == "contiguous":
+            h["m_indices"] = torch.from_numpy(c["m_indices"]).pin_memory()
+        host.append(h)
+    outs = [torch.empty(tuple(devs[0][i]["C"].shape), dtype=torch.bfloat16).pin_memory() for i in range(len(cases))]
+    h2d = sum(sum(t.numel() * t.element_size() for t in h.values()) for h in host)
+    d2h = sum(o.numel() * o.element_size() for o in outs)
+
+    def e2e_step():
+        for c, h, d, o in zip(cases, host, devs[0], outs):
+            for key, t in h.items():
+                d[key].copy_(t, non_blocking=True)
+            call(fg, c, d, stream=stream)
+            o.copy_(d["C"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    barrier(world, local)
+    e2e_value = step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)",
+            "data": "synthetic",
+            "config": {"workload": name, "shapes": [w["name"] for w in wl],
+                       "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
+                       "graph": "each step replayed from a CUDA graph", "parallelism": f"replicas x{world}"},
+            "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
+            "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
+            "roofline": roof,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks.summary(t_wall0, t_wall1), "device_status": fg.STATUS_NAMES.get(status, status)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s, f, cores = time_oracle(cases, row_fraction=1.0)
+        line["cpu_baseline"] = {"value": round(f / s / 1e12, 5), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                "sample": f"one full step of the {name} workload (every GEMM, all rows), {s:.1f} s"}
+    del graphs, egraphs
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default="decode_sweep")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

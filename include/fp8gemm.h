@@ -29,8 +29,8 @@
  *   B    : e4m3 codes, [N, K] (dense) or [G, N, K] (grouped).
  *   sfb  : fp32, [ceil(N/128), ceil(K/128)] (dense) or [G, ceil(N/128), ceil(K/128)].
  *   C    : bf16, [M, N] (dense / contiguous) or [G, Mmax, N] (masked).
- * Requirements: K % 16 == 0 and N % 8 == 0 (16-byte row strides); A, B, C
- * 16-byte aligned; sfa, sfb 4-byte aligned; K may end in a partial block.
+ * Requirements: K % 16 == 0 and N % 8 == 0 (16-byte row strides); A, B, C and
+ * sfa 16-byte aligned; sfb 4-byte aligned; K may end in a partial block.
  *
  * Ownership: the caller owns every buffer.  The library allocates only in
  * fg_init (a status word, a split-K workspace and its counters), never inside

@@ -47,6 +47,8 @@ constexpr int kMmaWarp = 9;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, far above any legal wait
 constexpr int kErrTimeout = 6;       // FG_ERR_TIMEOUT
 constexpr int kMaskedMaxGroups = 1024;
+constexpr int kSwapScaleBytes = 24 * 1024;  // shared memory for staged combined scales (swap kernel)
+constexpr int kScaleChunk = 16;             // K blocks per staged scale chunk (tiled kernel)
 
 enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
@@ -155,27 +157,69 @@ __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* 
   return ti;
 }
 
+// Combined scales of one chunk of kScaleChunk K blocks of a 128-row tile,
+// s[kb][row] = sfa[kb][m0+row] * sfb[nb][kb], as held in registers by one
+// promotion thread (thread tid covers K block tid/16 and rows (tid%16)*8 .. +8).
+struct ScaleChunkRegs {
+  float v[8];
+};
+
+template <int MODE>
+__device__ __forceinline__ void load_scale_chunk(const TiledParams& p, const TileInfo& ti, int chunk, int tid,
+                                                 ScaleChunkRegs& r) {
+  const int kb = chunk * kScaleChunk + tid / 16;
+  const int r8 = (tid % 16) * 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) r.v[i] = 0.0f;
+  if (kb >= p.num_kb) return;
+  const int nb = ti.n0 / kBlockK;
+  const size_t g_sfb = (MODE == kDense) ? 0 : static_cast<size_t>(ti.g);
+  const float sb = __ldg(p.sfb + (g_sfb * p.num_nb + nb) * p.num_kb + kb);
+  const size_t g_sfa = (MODE == kMasked) ? static_cast<size_t>(ti.g) : 0;
+  const float* sa = p.sfa + (g_sfa * p.num_kb + kb) * static_cast<size_t>(p.ld) + ti.m0 + r8;
+  const int rows_left = p.M - (ti.m0 + r8);  // rows of the row space from this thread's first row on
+  if (rows_left >= 8) {
+    const float4 a0 = __ldg(reinterpret_cast<const float4*>(sa));
+    const float4 a1 = __ldg(reinterpret_cast<const float4*>(sa) + 1);
+    r.v[0] = a0.x * sb; r.v[1] = a0.y * sb; r.v[2] = a0.z * sb; r.v[3] = a0.w * sb;
+    r.v[4] = a1.x * sb; r.v[5] = a1.y * sb; r.v[6] = a1.z * sb; r.v[7] = a1.w * sb;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (i < rows_left) r.v[i] = __ldg(sa + i) * sb;
+  }
+}
+
+__device__ __forceinline__ void store_scale_chunk(float* buf, int tid, const ScaleChunkRegs& r) {
+  float4* dst = reinterpret_cast<float4*>(buf + (tid / 16) * kBlockM + (tid % 16) * 8);
+  dst[0] = make_float4(r.v[0], r.v[1], r.v[2], r.v[3]);
+  dst[1] = make_float4(r.v[4], r.v[5], r.v[6], r.v[7]);
+}
+
 template <int BN, int STAGES, int NUM_TBUF, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const TiledParams p) {
-  static_assert(BN == 128 || BN == 256, "BN");
+  static_assert(BN == 128, "one 128-wide block of B scales per tile");
   constexpr int A_BYTES = kBlockM * kBlockK;
   constexpr int B_BYTES = BN * kBlockK;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t TMEM_COLS = NUM_TBUF * BN;
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   constexpr int COLS = BN / 2;  // columns per promotion thread
+  constexpr int CHUNK_FLOATS = kScaleChunk * kBlockM;
   constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, BN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  float* s_scale = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [2][kScaleChunk][128]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + 2 * CHUNK_FLOATS);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + NUM_TBUF;
   uint64_t* mma_done = tempty + NUM_TBUF;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* pbar = mma_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
 
@@ -186,36 +230,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
     mbar_init(mma_done, 1);
+    mbar_init(pbar, kPromoWarps * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == kProducerWarp && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
   if (warp == kMmaWarp) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
-  if (MODE == kMasked && warp == 0) {
-    // live 128-row blocks per group, exclusive prefix in s_prefix[0..G]
-    int carry = 0;
-    if (lane == 0) s_prefix[0] = 0;
-    for (int base = 0; base < p.G; base += 32) {
-      const int g = base + lane;
-      int v = 0;
-      if (g < p.G) {
-        int cnt = __ldg(p.masked_m + g);
-        cnt = cnt < 0 ? 0 : (cnt > p.M ? p.M : cnt);
-        v = (cnt + kBlockM - 1) / kBlockM;
-      }
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-      }
-      if (g < p.G) s_prefix[g + 1] = carry + v;
-      carry += __shfl_sync(0xffffffffu, v, 31);
-    }
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above overlaps the previous kernel's tail; from here on global memory is touched.
+  pdl_wait_prior_grid();
+  pdl_launch_dependents();
+
+  if (MODE == kMasked) {
+    if (warp == 0) {
+      // live 128-row blocks per group, exclusive prefix in s_prefix[0..G]
+      int carry = 0;
+      if (lane == 0) s_prefix[0] = 0;
+      for (int base = 0; base < p.G; base += 32) {
+        const int g = base + lane;
+        int v = 0;
+        if (g < p.G) {
+          int cnt = __ldg(p.masked_m + g);
+          cnt = cnt < 0 ? 0 : (cnt > p.M ? p.M : cnt);
+          v = (cnt + kBlockM - 1) / kBlockM;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (g < p.G) s_prefix[g + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+    }
+    __syncthreads();
+  }
 
   int num_tiles, live_mblocks = 1;
   if (MODE == kMasked) {
@@ -284,65 +336,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int h = warp >> 2;
     const int row = q * 32 + lane;
+    const int tid = threadIdx.x;  // 0..255 among promotion threads
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    uint32_t tb = 0, tphase = 0;
+    const int n_chunks = (p.num_kb + kScaleChunk - 1) / kScaleChunk;
+    uint32_t tb = 0, tphase = 0, pphase = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-      const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
-      if (!ti.live) continue;
-      const int m = ti.m0 + row;
-      int row_limit;                 // rows of this tile's row space that exist
-      const float* sa_ptr;
-      if (MODE == kMasked) {
-        row_limit = p.M;
-        sa_ptr = p.sfa + static_cast<size_t>(ti.g) * p.num_kb * p.ld + m;
-      } else {
-        row_limit = p.M;
-        sa_ptr = p.sfa + m;
+
+    // first live tile of this CTA
+    int t = blockIdx.x;
+    TileInfo ti;
+    ti.live = 0;
+    for (; t < num_tiles; t += gridDim.x) {
+      ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+      if (ti.live) break;
+    }
+    // Scale chunks form one sequence over this CTA's tiles; chunk X lives in s_scale[X % 2].
+    // The registers hold the chunk after the one being processed; it is stored into the other
+    // slot once this chunk is done, which is safe because the barrier that ended the previous
+    // chunk guarantees that no thread still reads that slot.
+    ScaleChunkRegs nxt;
+    int buf = 0;
+    if (t < num_tiles) {
+      load_scale_chunk<MODE>(p, ti, 0, tid, nxt);
+      store_scale_chunk(s_scale, tid, nxt);
+      ok = group_sync(pbar, pphase, abort_flag);
+    }
+    while (t < num_tiles && ok) {
+      // the tile after this one (for the chunk prefetch that crosses tiles)
+      int t_next = t + gridDim.x;
+      TileInfo ti_next;
+      ti_next.live = 0;
+      for (; t_next < num_tiles; t_next += gridDim.x) {
+        ti_next = tiled_tile<MODE>(p, s_prefix, live_mblocks, t_next, BN);
+        if (ti_next.live) break;
       }
-      const bool row_ok = m < row_limit;
-      const int nb = (ti.n0 + h * COLS) / kBlockK;
-      const float* sb_ptr = p.sfb + (static_cast<size_t>(MODE == kDense ? 0 : ti.g) * p.num_nb + nb) * p.num_kb;
+      const int m = ti.m0 + row;
 
       float acc[COLS];
 #pragma unroll
       for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
 
-      float sa_next = row_ok ? __ldg(sa_ptr) : 0.0f;
-      float sb_next = __ldg(sb_ptr);
-      for (int kb = 0; kb < p.num_kb; ++kb) {
-        const float sa = sa_next, sb = sb_next;
-        if (kb + 1 < p.num_kb) {
-          sa_next = row_ok ? __ldg(sa_ptr + static_cast<size_t>(kb + 1) * p.ld) : 0.0f;
-          sb_next = __ldg(sb_ptr + kb + 1);
-        }
-        if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        const float s = sa * sb;
-        const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
-#pragma unroll
-        for (int c0 = 0; c0 < COLS; c0 += 64) {
+      for (int c = 0; c < n_chunks && ok; ++c) {
+        // prefetch the next chunk of the sequence into registers
+        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, nxt);
+        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, nxt);
+        const float* sc = s_scale + buf * CHUNK_FLOATS + row;
+        const int kb_end = (c + 1) * kScaleChunk < p.num_kb ? (c + 1) * kScaleChunk : p.num_kb;
+        for (int kb = c * kScaleChunk; kb < kb_end; ++kb) {
+          const float s = sc[(kb - c * kScaleChunk) * kBlockM];
+          if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
           uint32_t v0[32], v1[32];
-          tmem_ld_32x32b_x32(taddr + c0, v0);
-          tmem_ld_32x32b_x32(taddr + c0 + 32, v1);
+          tmem_ld_32x32b_x32(taddr, v0);
+          tmem_ld_32x32b_x32(taddr + 32, v1);
           tmem_wait_ld();
-          if (c0 + 64 >= COLS) {  // whole slice read: hand the TMEM buffer back to the MMA
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[tb]);
-          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);  // hand the TMEM buffer back to the MMA
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            acc[c0 + j] = fmaf(__uint_as_float(v0[j]), s, acc[c0 + j]);
-            acc[c0 + 32 + j] = fmaf(__uint_as_float(v1[j]), s, acc[c0 + 32 + j]);
+            acc[j] = fmaf(__uint_as_float(v0[j]), s, acc[j]);
+            acc[32 + j] = fmaf(__uint_as_float(v1[j]), s, acc[32 + j]);
           }
+          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }
-        if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+        if (!ok) break;
+        // publish the prefetched chunk into the other slot, then one barrier
+        const int nbuf = buf ^ 1;
+        if (c + 1 < n_chunks || t_next < num_tiles) store_scale_chunk(s_scale + nbuf * CHUNK_FLOATS, tid, nxt);
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        buf = nbuf;
       }
       if (!ok) break;
 
       // epilogue: bf16 round-to-nearest-even, 16-byte stores of this thread's row segment
-      bool store_row = row_ok;
+      bool store_row = m < p.M;
       __nv_bfloat16* crow;
       if (MODE == kMasked) {
         int cnt = __ldg(p.masked_m + ti.g);
@@ -367,6 +436,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      t = t_next;
+      ti = ti_next;
     }
   }
 
@@ -387,6 +458,11 @@ __device__ __forceinline__ int sk_owner(long long u, int P, long long U) {
   return static_cast<int>(((u + 1) * P - 1) / U);
 }
 __device__ __forceinline__ long long sk_begin(int c, int P, long long U) { return (c * U) / P; }
+// Workspace slot of CTA c's piece of the tile whose first unit is tu0: slot 2c holds the
+// first segment of the CTA's range, slot 2c+1 its last (middle segments are whole tiles).
+__device__ __forceinline__ int sk_slot(int c, int P, long long U, long long tu0) {
+  return 2 * c + (sk_begin(c, P, U) >= tu0 ? 0 : 1);
+}
 
 template <int MP, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -399,14 +475,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NUM_TBUF = 4;
   constexpr uint32_t TMEM_COLS = (NUM_TBUF * MP) < 32 ? 32 : NUM_TBUF * MP;
   constexpr int COLS = MP / 2;                // token columns per promotion thread
-  constexpr int SFA_CHUNK = 32;               // K blocks of token scales staged at once
+  constexpr int SCALE_CAP = kSwapScaleBytes / (4 * MP);  // units whose scales fit in shared memory
+  constexpr int F4 = MP * kBlockM / 4 / (kPromoWarps * 32);  // float4 of a partial tile per thread
+  constexpr int PPR = (16 / F4) < 1 ? 1 : 16 / F4;             // partials read per round in the fix-up
   constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, MP);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   __nv_bfloat16* s_c = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * STAGE_BYTES);  // [MP][128]
-  float* s_sfa = reinterpret_cast<float*>(s_c + MP * kBlockM);                          // [SFA_CHUNK][MP]
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_sfa + SFA_CHUNK * MP);
+  float* s_scale = reinterpret_cast<float*>(s_c + MP * kBlockM);                        // [SCALE_CAP][MP]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + SCALE_CAP * MP);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + NUM_TBUF;
@@ -438,6 +516,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above overlaps the previous kernel's tail; from here on global memory is touched.
+  pdl_wait_prior_grid();
+  pdl_launch_dependents();
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
@@ -446,21 +527,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint64_t issued = 0;
       bool ok = true;
-      for (long long u = u_begin; u < u_end && ok;) {
+      for (long long u = u_begin; u < u_end && ok; ++u) {
         const int t = static_cast<int>(u / KB);
-        const int kb0 = static_cast<int>(u - static_cast<long long>(t) * KB);
-        const long long tile_end = static_cast<long long>(t + 1) * KB;
-        const int kb1 = static_cast<int>((u_end < tile_end ? u_end : tile_end) - static_cast<long long>(t) * KB);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          uint8_t* sw = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_2d(sw, &tmW, &full[stage], kb * kBlockK, t * kBlockM, pol_w);
-          tma_load_2d(sw + W_BYTES, &tmT, &full[stage], kb * kBlockK, 0, pol_t);
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        }
-        u = static_cast<long long>(t) * KB + kb1;
+        const int kb = static_cast<int>(u - static_cast<long long>(t) * KB);
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        uint8_t* sw = smem + stage * STAGE_BYTES;
+        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+        tma_load_2d(sw, &tmW, &full[stage], kb * kBlockK, t * kBlockM, pol_w);
+        tma_load_2d(sw + W_BYTES, &tmT, &full[stage], kb * kBlockK, 0, pol_t);
+        ++issued;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
       if (!ok) {
         const uint64_t first = issued > STAGES ? issued - STAGES : 0;
@@ -471,29 +547,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
-      bool ok = true;
-      for (long long u = u_begin; u < u_end && ok;) {
-        const int t = static_cast<int>(u / KB);
-        const int kb0 = static_cast<int>(u - static_cast<long long>(t) * KB);
-        const long long tile_end = static_cast<long long>(t + 1) * KB;
-        const int kb1 = static_cast<int>((u_end < tile_end ? u_end : tile_end) - static_cast<long long>(t) * KB);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t d = tmem_base + tb * MP;
-          const uint32_t sw = smem_addr(smem + stage * STAGE_BYTES);
-          const uint64_t adesc = smem_desc_k128_sw128(sw);
-          const uint64_t bdesc = smem_desc_k128_sw128(sw + W_BYTES);
+      for (long long u = u_begin; u < u_end; ++u) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
+        if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + tb * MP;
+        const uint32_t sw = smem_addr(smem + stage * STAGE_BYTES);
+        const uint64_t adesc = smem_desc_k128_sw128(sw);
+        const uint64_t bdesc = smem_desc_k128_sw128(sw + W_BYTES);
 #pragma unroll
-          for (int j = 0; j < kBlockK / 32; ++j)
-            mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
-          mma_commit(&empty[stage]);
-          mma_commit(&tfull[tb]);
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
-        }
-        u = static_cast<long long>(t) * KB + kb1;
+        for (int j = 0; j < kBlockK / 32; ++j)
+          mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+        mma_commit(&empty[stage]);
+        mma_commit(&tfull[tb]);
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
       }
       mma_commit(mma_done);
       mbar_drain(mma_done, 0);
@@ -508,30 +576,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tb = 0, tphase = 0, pphase = 0;
     bool ok = true;
     bool first_segment = true;
+    long long chunk_base = u_begin, chunk_end = u_begin;  // units whose scales are staged
     for (long long u = u_begin; u < u_end && ok;) {
       const int t = static_cast<int>(u / KB);
-      const int kb0 = static_cast<int>(u - static_cast<long long>(t) * KB);
-      const long long tile_end = static_cast<long long>(t + 1) * KB;
-      const int kb1 = static_cast<int>((u_end < tile_end ? u_end : tile_end) - static_cast<long long>(t) * KB);
-      const float* sb_ptr = p.sfb + static_cast<size_t>(t) * KB;
+      const long long tu0 = static_cast<long long>(t) * KB;
+      const int kb0 = static_cast<int>(u - tu0);
+      const int kb1 = static_cast<int>((u_end < tu0 + KB ? u_end : tu0 + KB) - tu0);
 
       float acc[COLS];
 #pragma unroll
       for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
 
-      int chunk0 = -1;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (kb >= chunk0 + SFA_CHUNK || chunk0 < 0) {
-          // stage token scales sfa[kb..kb+SFA_CHUNK)[0..MP) (zero past M)
+        const long long uu = tu0 + kb;
+        if (uu >= chunk_end) {
+          // combined scales sfa[kb][m] * sfb[t][kb] of the next SCALE_CAP units (zero past M)
           if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
-          chunk0 = kb;
-          for (int i = tid; i < SFA_CHUNK * MP; i += kPromoWarps * 32) {
-            const int kk = chunk0 + i / MP, mm = i % MP;
-            s_sfa[i] = (kk < kb1 && mm < p.M) ? __ldg(p.sfa + static_cast<size_t>(kk) * p.ld + mm) : 0.0f;
+          chunk_base = uu;
+          chunk_end = (u_end < uu + SCALE_CAP) ? u_end : uu + SCALE_CAP;
+          const int n = static_cast<int>(chunk_end - chunk_base) * MP;
+#pragma unroll 4
+          for (int i = tid; i < n; i += kPromoWarps * 32) {
+            const long long v = chunk_base + i / MP;
+            const int mm = i % MP;
+            const int vt = static_cast<int>(v / KB);
+            const int vkb = static_cast<int>(v - static_cast<long long>(vt) * KB);
+            s_scale[i] = (mm < p.M) ? __ldg(p.sfa + static_cast<size_t>(vkb) * p.ld + mm) *
+                                          __ldg(p.sfb + static_cast<size_t>(vt) * KB + vkb)
+                                    : 0.0f;
           }
           if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
         }
-        const float sb = __ldg(sb_ptr + kb);
         if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
         tc_fence_after();
         const uint32_t taddr = tmem_base + lane_off + tb * MP + h * COLS;
@@ -550,70 +625,96 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tempty[tb]);
-        const float4* sf4 = reinterpret_cast<const float4*>(s_sfa + (kb - chunk0) * MP + h * COLS);
+        const float4* sc4 = reinterpret_cast<const float4*>(s_scale + (uu - chunk_base) * MP + h * COLS);
 #pragma unroll
         for (int j = 0; j < COLS; j += 4) {
-          const float4 a4 = sf4[j / 4];
-          acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), a4.x * sb, acc[j + 0]);
-          acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), a4.y * sb, acc[j + 1]);
-          acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), a4.z * sb, acc[j + 2]);
-          acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), a4.w * sb, acc[j + 3]);
+          const float4 s4 = sc4[j / 4];
+          acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), s4.x, acc[j + 0]);
+          acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), s4.y, acc[j + 1]);
+          acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), s4.z, acc[j + 2]);
+          acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), s4.w, acc[j + 3]);
         }
         if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
       }
       if (!ok) break;
 
-      const bool whole = (kb0 == 0 && kb1 == KB);
-      bool do_store = whole;
-      if (!whole) {
-        // publish this CTA's partial, then let the last of the tile's CTAs sum them
-        const int slot = 2 * blockIdx.x + (first_segment ? 0 : 1);
-        float* wp = p.ws + static_cast<size_t>(slot) * MP * kBlockM + nl;
-#pragma unroll
-        for (int j = 0; j < COLS; ++j) wp[static_cast<size_t>(h * COLS + j) * kBlockM] = acc[j];
-        __threadfence();
-        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
-        const long long tu0 = static_cast<long long>(t) * KB;
-        const int c_first = sk_owner(tu0, P, U);
-        const int c_last = sk_owner(tu0 + KB - 1, P, U);
-        if (tid == 0) {
-          const int prev = atomicAdd(p.counters + t, 1);
-          const int last = (prev == c_last - c_first);
-          if (last) p.counters[t] = 0;  // ready for the next launch
-          *s_last = last;
-        }
-        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
-        if (*s_last) {
-          __threadfence();
-#pragma unroll
-          for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
-          for (int c = c_first; c <= c_last; ++c) {
-            const int cs = 2 * c + (sk_begin(c, P, U) >= tu0 ? 0 : 1);
-            const float* rp = p.ws + static_cast<size_t>(cs) * MP * kBlockM + nl;
-#pragma unroll
-            for (int j = 0; j < COLS; ++j) acc[j] += __ldcg(rp + static_cast<size_t>(h * COLS + j) * kBlockM);
-          }
-          do_store = true;
-        }
-      }
-      if (do_store) {
-        // transpose through shared memory: s_c[m][nl], then 16-byte row stores of C[m, t*128 ..]
+      const int n_base = t * kBlockM;
+      if (kb0 == 0 && kb1 == KB) {
+        // whole tile: transpose through shared memory, s_c[m][nl], then 16-byte row stores of C
 #pragma unroll
         for (int j = 0; j < COLS; ++j) s_c[(h * COLS + j) * kBlockM + nl] = __float2bfloat16_rn(acc[j]);
         if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
         const int rows = p.M < MP ? p.M : MP;
-        const int n_base = t * kBlockM;
         for (int i = tid; i < rows * (kBlockM / 8); i += kPromoWarps * 32) {
           const int mm = i / (kBlockM / 8), ch = i % (kBlockM / 8);
           if (n_base + ch * 8 < p.N) {
-            const uint4 v = *reinterpret_cast<const uint4*>(s_c + mm * kBlockM + ch * 8);
-            *reinterpret_cast<uint4*>(p.C + static_cast<size_t>(mm) * p.N + n_base + ch * 8) = v;
+            const uint4 val = *reinterpret_cast<const uint4*>(s_c + mm * kBlockM + ch * 8);
+            *reinterpret_cast<uint4*>(p.C + static_cast<size_t>(mm) * p.N + n_base + ch * 8) = val;
           }
         }
         if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+      } else {
+        // split tile: publish this CTA's fp32 partial; the last of the tile's CTAs to arrive sums
+        // all partials in CTA order (deterministic) and writes the bf16 tile
+        const int slot = 2 * blockIdx.x + (first_segment ? 0 : 1);
+        float* wp = p.ws + static_cast<size_t>(slot) * MP * kBlockM + nl;
+#pragma unroll
+        for (int j = 0; j < COLS; ++j) wp[static_cast<size_t>(h * COLS + j) * kBlockM] = acc[j];
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        const int c_first = sk_owner(tu0, P, U);
+        const int c_last = sk_owner(tu0 + KB - 1, P, U);
+        if (tid == 0) {
+          fence_acq_rel_gpu();  // release the partials written by this CTA (ordered by the barrier)
+          const int prev = atomicAdd(p.counters + t, 1);
+          const int last = (prev == c_last - c_first);
+          if (last) {
+            fence_acq_rel_gpu();  // acquire the other CTAs' partials
+            p.counters[t] = 0;    // ready for the next launch
+          }
+          *s_last = last;
+        }
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        if (*s_last) {
+          const float4* ws4 = reinterpret_cast<const float4*>(p.ws);
+          float4 r[F4];
+#pragma unroll
+          for (int i = 0; i < F4; ++i) r[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int c0 = c_first; c0 <= c_last; c0 += PPR) {
+            float4 a[PPR][F4];
+#pragma unroll
+            for (int k = 0; k < PPR; ++k) {
+              if (c0 + k <= c_last) {
+                const float4* src = ws4 + static_cast<size_t>(sk_slot(c0 + k, P, U, tu0)) * (MP * kBlockM / 4) + tid;
+#pragma unroll
+                for (int i = 0; i < F4; ++i) a[k][i] = __ldcg(src + i * kPromoWarps * 32);
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < PPR; ++k) {
+              if (c0 + k <= c_last) {
+#pragma unroll
+                for (int i = 0; i < F4; ++i) {
+                  r[i].x += a[k][i].x; r[i].y += a[k][i].y; r[i].z += a[k][i].z; r[i].w += a[k][i].w;
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < F4; ++i) {
+            const int f = tid + i * kPromoWarps * 32;  // float4 index in the [MP][128] tile
+            const int mm = f >> 5;
+            const int n = n_base + (f & 31) * 4;
+            if (mm < p.M && n < p.N) {
+              uint2 val;
+              val.x = pack_bf16x2(r[i].x, r[i].y);
+              val.y = pack_bf16x2(r[i].z, r[i].w);
+              *reinterpret_cast<uint2*>(p.C + static_cast<size_t>(mm) * p.N + n) = val;
+            }
+          }
+        }
       }
       first_segment = false;
-      u = static_cast<long long>(t) * KB + kb1;
+      u = tu0 + kb1;
     }
   }
 

@@ -47,7 +47,8 @@ constexpr int kTiledTbuf = 4;
 
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
-  return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBlockM + BN) * kBlockK + 256 /*barriers*/ +
+  return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBlockM + BN) * kBlockK +
+         2 * fg::kScaleChunk * kBlockM * 4 /*scale chunks*/ + 256 /*barriers*/ +
          4 * (fg::kMaskedMaxGroups + 1) /*masked prefix*/;
 }
 
@@ -59,7 +60,7 @@ constexpr int swap_stages() {
 template <int MP, int STAGES>
 constexpr size_t swap_smem_bytes() {
   return 1024 + static_cast<size_t>(STAGES) * (kBlockM + MP) * kBlockK + MP * kBlockM * 2 /*C staging*/ +
-         32 * MP * 4 /*token scales*/ + 256 /*barriers*/;
+         fg::kSwapScaleBytes /*combined scales*/ + 256 /*barriers*/;
 }
 
 int current_device() {
@@ -121,14 +122,20 @@ fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap&
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
   void* args[3] = {const_cast<CUtensorMap*>(&m0), const_cast<CUtensorMap*>(&m1), const_cast<void*>(params_ptr)};
+  // programmatic dependent launch: the kernel's prologue (barriers, TMEM allocation, descriptor
+  // prefetch) may overlap the previous kernel of the stream; the kernel waits for that kernel
+  // (griddepcontrol.wait) before its first global-memory access
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = grid;
   cfg.blockDim = dim3(fg::kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cfg.attrs = nullptr;
-  cfg.numAttrs = 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(kernel), args);
   if (e != cudaSuccess) return FG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -141,7 +148,7 @@ fg_status check_common(const void* A, const float* sfa, const void* B, const flo
   if (!A || !sfa || !B || !sfb || !C) return FG_ERR_INVALID_ARG;
   if (N < 0 || K <= 0) return FG_ERR_INVALID_ARG;
   if (K % 16 != 0 || N % 8 != 0) return FG_ERR_ALIGNMENT;
-  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sfa, 4) || !aligned(sfb, 4))
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(sfa, 16) || !aligned(sfb, 4))
     return FG_ERR_ALIGNMENT;
   return FG_OK;
 }
