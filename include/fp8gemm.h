@@ -32,6 +32,9 @@
  * Requirements: K % 16 == 0 and N % 8 == 0 (16-byte row strides); A, B, C and
  * sfa 16-byte aligned; sfb 4-byte aligned; K may end in a partial block.
  *
+ * Results are deterministic: repeated calls on the same inputs give
+ * bit-identical outputs (split-K partials are summed in a fixed order).
+ *
  * Ownership: the caller owns every buffer.  The library allocates only in
  * fg_init (a status word, a split-K workspace and its counters), never inside
  * a GEMM call, so calls can be captured into CUDA graphs.  The workspace is

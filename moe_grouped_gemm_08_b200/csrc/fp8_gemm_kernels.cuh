@@ -226,7 +226,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) {
+  // Producer state (lane 0 of the producer warp): tile walk position, smem ring position, loads issued.
+  int p_t = blockIdx.x, p_kb = 0;
+  TileInfo p_ti;
+  p_ti.live = 0;
+  uint32_t p_stage = 0, p_phase = 0;
+  uint64_t p_issued = 0;
+  const bool producer = (warp == kProducerWarp && lane == 0);
+  auto issue = [&](const TileInfo& ti, int kb) {
+    uint8_t* sa = smem + p_stage * STAGE_BYTES;
+    mbar_arrive_expect_tx(&full[p_stage], STAGE_BYTES);
+    tma_load_3d(sa, &tmA, &full[p_stage], kb * kBlockK, ti.m0, (MODE == kMasked) ? ti.g : 0);
+    tma_load_3d(sa + A_BYTES, &tmB, &full[p_stage], kb * kBlockK, ti.n0, (MODE == kDense) ? 0 : ti.g);
+    ++p_issued;
+    if (++p_stage == STAGES) { p_stage = 0; p_phase ^= 1u; }
+  };
+
+  if (producer) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
     mbar_init(mma_done, 1);
@@ -234,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); }
   if (warp == kMmaWarp) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -279,27 +296,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      uint64_t issued = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
-        if (!ti.live) continue;
-        const int ga = (MODE == kMasked) ? ti.g : 0;
-        const int gb = (MODE == kDense) ? 0 : ti.g;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-          uint8_t* sa = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_3d(sa, &tmA, &full[stage], kb * kBlockK, ti.m0, ga);
-          tma_load_3d(sa + A_BYTES, &tmB, &full[stage], kb * kBlockK, ti.n0, gb);
-          ++issued;
-          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      for (; p_t < num_tiles; p_t += gridDim.x) {  // this CTA's first live tile
+        p_ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, p_t, BN);
+        if (p_ti.live) break;
+      }
+      while (p_t < num_tiles) {
+        if (!mbar_wait(&empty[p_stage], p_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        issue(p_ti, p_kb);
+        if (++p_kb == p.num_kb) {
+          p_kb = 0;
+          for (p_t += gridDim.x; p_t < num_tiles; p_t += gridDim.x) {
+            p_ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, p_t, BN);
+            if (p_ti.live) break;
+          }
         }
       }
       if (!ok) {  // drain this CTA's copies still in flight before the CTA exits
-        const uint64_t first = issued > STAGES ? issued - STAGES : 0;
-        for (uint64_t i = first; i < issued; ++i)
+        const uint64_t first = p_issued > STAGES ? p_issued - STAGES : 0;
+        for (uint64_t i = first; i < p_issued; ++i)
           mbar_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
       }
     }
@@ -454,13 +469,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ============================================================================
 // Kernel 2: swap-AB stream-K (dense, M <= MP <= 128)
 // ============================================================================
-__device__ __forceinline__ int sk_owner(long long u, int P, long long U) {
-  return static_cast<int>(((u + 1) * P - 1) / U);
+// Units are (n-tile, K block) pairs, u = t * KB + kb; CTA c owns units [begin(c), begin(c+1)).
+// N * K < 2^40 keeps the unit count below 2^26, so unit indices fit in 32 bits.
+__device__ __forceinline__ int sk_begin(int c, int P, int U) {
+  return static_cast<int>((static_cast<long long>(c) * U) / P);
 }
-__device__ __forceinline__ long long sk_begin(int c, int P, long long U) { return (c * U) / P; }
-// Workspace slot of CTA c's piece of the tile whose first unit is tu0: slot 2c holds the
-// first segment of the CTA's range, slot 2c+1 its last (middle segments are whole tiles).
-__device__ __forceinline__ int sk_slot(int c, int P, long long U, long long tu0) {
+__device__ __forceinline__ int sk_owner(int u, int P, int U) {
+  return static_cast<int>(((static_cast<long long>(u) + 1) * P - 1) / U);
+}
+// Workspace slot of CTA c's piece of the tile whose first unit is tu0.
+// Slot 2c holds the first segment of the CTA's range, slot 2c+1 its last (middle segments are
+// whole tiles and never need a slot).
+__device__ __forceinline__ int sk_slot(int c, int P, int U, int tu0) {
   return 2 * c + (sk_begin(c, P, U) >= tu0 ? 0 : 1);
 }
 
@@ -475,9 +495,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int NUM_TBUF = 4;
   constexpr uint32_t TMEM_COLS = (NUM_TBUF * MP) < 32 ? 32 : NUM_TBUF * MP;
   constexpr int COLS = MP / 2;                // token columns per promotion thread
+  constexpr int NPROMO = kPromoWarps * 32;
   constexpr int SCALE_CAP = kSwapScaleBytes / (4 * MP);  // units whose scales fit in shared memory
-  constexpr int F4 = MP * kBlockM / 4 / (kPromoWarps * 32);  // float4 of a partial tile per thread
-  constexpr int PPR = (16 / F4) < 1 ? 1 : 16 / F4;             // partials read per round in the fix-up
+  constexpr int F4 = MP * kBlockM / 4 / NPROMO;          // float4 of a partial tile per thread
+  constexpr int PPR = (16 / F4) < 1 ? 1 : 16 / F4;       // partials read per round in the fix-up
   constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, MP);
 
   extern __shared__ uint8_t smem_raw[];
@@ -498,19 +519,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int P = gridDim.x;
   const int KB = p.num_kb;
-  const long long U = static_cast<long long>(p.n_tiles) * KB;
-  const long long u_begin = sk_begin(blockIdx.x, P, U);
-  const long long u_end = sk_begin(blockIdx.x + 1, P, U);
+  const int U = p.n_tiles * KB;
+  const int u_begin = sk_begin(blockIdx.x, P, U);
+  const int u_end = sk_begin(blockIdx.x + 1, P, U);
 
-  if (threadIdx.x == 0) {
+  const uint64_t pol_w = l2_policy_evict_first();  // each weight byte is read once
+  const uint64_t pol_t = l2_policy_evict_last();   // tokens are re-read by every CTA
+  // Producer state: next unit to load, smem ring position, loads issued.
+  int p_u = u_begin;
+  uint32_t p_stage = 0, p_phase = 0;
+  uint32_t p_issued = 0;
+  auto issue = [&](int u) {
+    const int t = u / KB;
+    const int kb = u - t * KB;
+    uint8_t* sw = smem + p_stage * STAGE_BYTES;
+    mbar_arrive_expect_tx(&full[p_stage], STAGE_BYTES);
+    tma_load_2d(sw, &tmW, &full[p_stage], kb * kBlockK, t * kBlockM, pol_w);
+    tma_load_2d(sw + W_BYTES, &tmT, &full[p_stage], kb * kBlockK, 0, pol_t);
+    ++p_issued;
+    if (++p_stage == STAGES) { p_stage = 0; p_phase ^= 1u; }
+  };
+
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tmap(&tmW);
+    prefetch_tmap(&tmT);
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
     mbar_init(mma_done, 1);
-    mbar_init(pbar, kPromoWarps * 32);
+    mbar_init(pbar, NPROMO);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kProducerWarp && lane == 0) { prefetch_tmap(&tmW); prefetch_tmap(&tmT); }
   if (warp == kMmaWarp) { tmem_alloc(tmem_slot, TMEM_COLS); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
@@ -522,32 +561,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();  // each weight byte is read once
-      const uint64_t pol_t = l2_policy_evict_last();   // tokens are re-read by every CTA
-      uint32_t stage = 0, phase = 0;
-      uint64_t issued = 0;
       bool ok = true;
-      for (long long u = u_begin; u < u_end && ok; ++u) {
-        const int t = static_cast<int>(u / KB);
-        const int kb = static_cast<int>(u - static_cast<long long>(t) * KB);
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-        uint8_t* sw = smem + stage * STAGE_BYTES;
-        mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-        tma_load_2d(sw, &tmW, &full[stage], kb * kBlockK, t * kBlockM, pol_w);
-        tma_load_2d(sw + W_BYTES, &tmT, &full[stage], kb * kBlockK, 0, pol_t);
-        ++issued;
-        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      for (; p_u < u_end; ++p_u) {
+        if (!mbar_wait(&empty[p_stage], p_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+        issue(p_u);
       }
       if (!ok) {
-        const uint64_t first = issued > STAGES ? issued - STAGES : 0;
-        for (uint64_t i = first; i < issued; ++i)
-          mbar_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+        const uint32_t first = p_issued > STAGES ? p_issued - STAGES : 0;
+        for (uint32_t i = first; i < p_issued; ++i) mbar_drain(&full[i % STAGES], (i / STAGES) & 1u);
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
-      for (long long u = u_begin; u < u_end; ++u) {
+      for (int u = u_begin; u < u_end; ++u) {
         if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
         if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) break;
         tc_fence_after();
@@ -576,35 +603,64 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t tb = 0, tphase = 0, pphase = 0;
     bool ok = true;
     bool first_segment = true;
-    long long chunk_base = u_begin, chunk_end = u_begin;  // units whose scales are staged
-    for (long long u = u_begin; u < u_end && ok;) {
-      const int t = static_cast<int>(u / KB);
-      const long long tu0 = static_cast<long long>(t) * KB;
-      const int kb0 = static_cast<int>(u - tu0);
-      const int kb1 = static_cast<int>((u_end < tu0 + KB ? u_end : tu0 + KB) - tu0);
+    int chunk_base = u_begin, chunk_end = u_begin;  // units whose scales are staged
+
+    // bf16 tile from registers (thread = weight row nl, columns = tokens) -> C[m, t*128 + nl],
+    // transposed through shared memory so that the global stores are 16-byte row segments
+    auto store_tile = [&](const float* vals, int n_base) -> bool {
+#pragma unroll
+      for (int j = 0; j < COLS; ++j) s_c[(h * COLS + j) * kBlockM + nl] = __float2bfloat16_rn(vals[j]);
+      if (!group_sync(pbar, pphase, abort_flag)) return false;
+      const int rows = p.M < MP ? p.M : MP;
+      for (int i = tid; i < rows * (kBlockM / 8); i += NPROMO) {
+        const int mm = i / (kBlockM / 8), ch = i % (kBlockM / 8);
+        if (n_base + ch * 8 < p.N) {
+          const uint4 val = *reinterpret_cast<const uint4*>(s_c + mm * kBlockM + ch * 8);
+          *reinterpret_cast<uint4*>(p.C + static_cast<size_t>(mm) * p.N + n_base + ch * 8) = val;
+        }
+      }
+      return group_sync(pbar, pphase, abort_flag);
+    };
+
+    for (int u = u_begin; u < u_end && ok;) {
+      const int t = u / KB;
+      const int tu0 = t * KB;
+      const int kb0 = u - tu0;
+      const int kb1 = (u_end < tu0 + KB ? u_end : tu0 + KB) - tu0;
 
       float acc[COLS];
 #pragma unroll
       for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
 
       for (int kb = kb0; kb < kb1; ++kb) {
-        const long long uu = tu0 + kb;
+        const int uu = tu0 + kb;
         if (uu >= chunk_end) {
-          // combined scales sfa[kb][m] * sfb[t][kb] of the next SCALE_CAP units (zero past M)
+          // combined scales sfa[kb][m] * sfb[t][kb] of the next SCALE_CAP units (zero past M);
+          // thread tid owns column tid % MP of units tid / MP + r * (256 / MP), and every load
+          // of the chunk is issued before the first product is formed
           if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
           chunk_base = uu;
           chunk_end = (u_end < uu + SCALE_CAP) ? u_end : uu + SCALE_CAP;
-          const int n = static_cast<int>(chunk_end - chunk_base) * MP;
-#pragma unroll 4
-          for (int i = tid; i < n; i += kPromoWarps * 32) {
-            const long long v = chunk_base + i / MP;
-            const int mm = i % MP;
-            const int vt = static_cast<int>(v / KB);
-            const int vkb = static_cast<int>(v - static_cast<long long>(vt) * KB);
-            s_scale[i] = (mm < p.M) ? __ldg(p.sfa + static_cast<size_t>(vkb) * p.ld + mm) *
-                                          __ldg(p.sfb + static_cast<size_t>(vt) * KB + vkb)
-                                    : 0.0f;
+          constexpr int STEP = NPROMO / MP;  // units per pass of all threads
+          constexpr int ITER = SCALE_CAP / STEP;
+          const int mm = tid % MP;
+          const int v0 = chunk_base + tid / MP;
+          int vt = v0 / KB;
+          int vkb = v0 - vt * KB;
+          float a[ITER], b[ITER];
+#pragma unroll
+          for (int r = 0; r < ITER; ++r) {
+            a[r] = 0.0f;
+            b[r] = 0.0f;
+            if (v0 + r * STEP < chunk_end) {
+              if (mm < p.M) a[r] = __ldg(p.sfa + static_cast<size_t>(vkb) * p.ld + mm);
+              b[r] = __ldg(p.sfb + static_cast<size_t>(vt) * KB + vkb);
+            }
+            vkb += STEP;
+            while (vkb >= KB) { vkb -= KB; ++vt; }
           }
+#pragma unroll
+          for (int r = 0; r < ITER; ++r) s_scale[(tid / MP + r * STEP) * MP + mm] = a[r] * b[r];
           if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
         }
         if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
@@ -639,32 +695,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
 
       const int n_base = t * kBlockM;
-      if (kb0 == 0 && kb1 == KB) {
-        // whole tile: transpose through shared memory, s_c[m][nl], then 16-byte row stores of C
-#pragma unroll
-        for (int j = 0; j < COLS; ++j) s_c[(h * COLS + j) * kBlockM + nl] = __float2bfloat16_rn(acc[j]);
-        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
-        const int rows = p.M < MP ? p.M : MP;
-        for (int i = tid; i < rows * (kBlockM / 8); i += kPromoWarps * 32) {
-          const int mm = i / (kBlockM / 8), ch = i % (kBlockM / 8);
-          if (n_base + ch * 8 < p.N) {
-            const uint4 val = *reinterpret_cast<const uint4*>(s_c + mm * kBlockM + ch * 8);
-            *reinterpret_cast<uint4*>(p.C + static_cast<size_t>(mm) * p.N + n_base + ch * 8) = val;
-          }
-        }
-        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+      if (kb0 == 0 && kb1 == KB) {  // whole tile
+        if (!store_tile(acc, n_base)) { ok = false; break; }
       } else {
-        // split tile: publish this CTA's fp32 partial; the last of the tile's CTAs to arrive sums
-        // all partials in CTA order (deterministic) and writes the bf16 tile
+        // split tile: the CTAs of the tile publish their fp32 partials; the last to arrive
+        // (counter per tile) sums them in CTA order -- so results are bit-reproducible -- and
+        // writes the bf16 tile.  No CTA ever waits for another.
+        const int c_first = sk_owner(tu0, P, U);
+        const int c_last = sk_owner(tu0 + KB - 1, P, U);
         const int slot = 2 * blockIdx.x + (first_segment ? 0 : 1);
         float* wp = p.ws + static_cast<size_t>(slot) * MP * kBlockM + nl;
 #pragma unroll
         for (int j = 0; j < COLS; ++j) wp[static_cast<size_t>(h * COLS + j) * kBlockM] = acc[j];
         if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
-        const int c_first = sk_owner(tu0, P, U);
-        const int c_last = sk_owner(tu0 + KB - 1, P, U);
         if (tid == 0) {
-          fence_acq_rel_gpu();  // release the partials written by this CTA (ordered by the barrier)
+          fence_acq_rel_gpu();  // release the CTA's partial (ordered before by the barrier)
           const int prev = atomicAdd(p.counters + t, 1);
           const int last = (prev == c_last - c_first);
           if (last) {
@@ -686,7 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (c0 + k <= c_last) {
                 const float4* src = ws4 + static_cast<size_t>(sk_slot(c0 + k, P, U, tu0)) * (MP * kBlockM / 4) + tid;
 #pragma unroll
-                for (int i = 0; i < F4; ++i) a[k][i] = __ldcg(src + i * kPromoWarps * 32);
+                for (int i = 0; i < F4; ++i) a[k][i] = __ldcg(src + i * NPROMO);
               }
             }
 #pragma unroll
@@ -701,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int i = 0; i < F4; ++i) {
-            const int f = tid + i * kPromoWarps * 32;  // float4 index in the [MP][128] tile
+            const int f = tid + i * NPROMO;  // float4 index in the [MP][128] tile
             const int mm = f >> 5;
             const int n = n_base + (f & 31) * 4;
             if (mm < p.M && n < p.N) {

@@ -30,7 +30,7 @@ struct DeviceState {
   bool ready = false;
   int sms = 0;
   int* status = nullptr;
-  float* ws = nullptr;
+  float* ws = nullptr;   // split-K partial tiles
   int* counters = nullptr;
 };
 
