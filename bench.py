@@ -80,7 +80,11 @@ def cdiv(a, b):
     return (a + b - 1) // b
 
 
-def workload_list(name: str):
+def workload_list(name: str, shape: str | None = None):
+    if shape:
+        M, N, K = (int(x) for x in shape.split(","))
+        return f"dense_M{M}_N{N}_K{K}", [dict(name=f"dense_M{M}_N{N}_K{K}", seed=77, M=M, N=N, K=K,
+                                              row_scaled=M <= 128)]
     table = {"decode_sweep": workloads.decode_sweep, "dense_single": workloads.dense_single,
              "prefill": workloads.prefill, "contiguous": workloads.contiguous, "masked": workloads.masked}
     if name not in table:
@@ -292,7 +296,7 @@ def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on the same workload, rank 0 only."""
     if rank != 0:
         return
-    name, wl = workload_list(args.workload)
+    name, wl = workload_list(args.workload, args.shape)
     cases = [make_case(w) for w in wl]
     full_flops = sum(work_of(c)[0] for c in cases)
     # size each step so that warm-up + timed steps stay within about two minutes
@@ -328,7 +332,7 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     fg.init(local)
-    name, wl = workload_list(args.workload)
+    name, wl = workload_list(args.workload, args.shape)
     cases = [make_case(w) for w in wl]
     works = [work_of(c) for c in cases]
     step_flops = sum(w[0] for w in works)
@@ -513,7 +517,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--workload", default="decode_sweep")
+    ap.add_argument("--workload", default="decode_sweep",
+                    help="decode_sweep (default), dense_single, prefill, contiguous or masked")
+    ap.add_argument("--shape", default=None, help="M,N,K: one dense GEMM instead of a workload (profiling)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
