@@ -105,6 +105,33 @@ fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B
                                   void* C, const int* masked_m, int G, int Mmax, int N, int K,
                                   void* stream);
 
+/* Allocation-free variant of fp8_gemm_nt, for callers that cannot allocate device
+ * memory: code running inside another framework's memory pool or a pre-planned
+ * static memory budget, code that must not touch the allocator during a
+ * latency-critical decode step, or a process that has reserved the whole device
+ * up front.  (The pages have no counterpart; it is a deployment convenience.)
+ * It takes the same arguments as fp8_gemm_nt, needs no fg_init, and never calls
+ * cudaMalloc or cudaFree: its split-K scratch (partial tiles, per-tile counters,
+ * a status word; 16 MiB + 64 KiB) is a static device array that every GPU which
+ * loads this library holds until the process exits.
+ * Limits: M <= 128 (the swap-AB stream-K kernel; larger M returns
+ * FG_ERR_UNSUPPORTED) and ceil(N / 128) <= 16384 (else FG_ERR_UNSUPPORTED); the
+ * array caps the grid at 16 MiB / (2 * 128 * MP * 4 bytes) CTAs, MP = M rounded
+ * up to 32, 64 or 128, so M > 64 runs on at most 128 CTAs.
+ * The first call on a device looks up the array's device address (and the
+ * tensor-map encoder); make that first call before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU (concurrent
+ * streams, or other host threads) race and give wrong results.  Each call clears
+ * the counters it uses (a memset on `stream`) before its kernel; the partial
+ * tiles keep the last call's contents, which no call reads before writing.
+ * A wait that times out inside this variant is reported by fg_noalloc_status. */
+fg_status fp8_gemm_nt_noalloc(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                              int M, int N, int K, void* stream);
+
+/* Synchronise `stream`, then read and clear the status word of the
+ * allocation-free variant (FG_OK if it was never called on this device). */
+fg_status fg_noalloc_status(void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word:
  * FG_OK, or FG_ERR_TIMEOUT if some kernel since the last call gave up a wait. */
 fg_status fg_get_device_status(void* stream);

@@ -42,6 +42,10 @@ _lib.fp8_gemm_grouped_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int,
 _lib.fp8_gemm_grouped_contiguous.restype = _int
 _lib.fp8_gemm_grouped_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
 _lib.fp8_gemm_grouped_masked.restype = _int
+_lib.fp8_gemm_nt_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
+_lib.fp8_gemm_nt_noalloc.restype = _int
+_lib.fg_noalloc_status.argtypes = [_vp]
+_lib.fg_noalloc_status.restype = _int
 _lib.fg_get_device_status.argtypes = [_vp]
 _lib.fg_get_device_status.restype = _int
 _lib.fg_status_string.argtypes = [_int]

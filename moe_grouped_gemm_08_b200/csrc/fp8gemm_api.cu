@@ -215,6 +215,83 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
                                                                mW, mT, &p);
 }
 
+// ---------------------------------------------------------------------------------------------
+// Allocation-free variant of the dense small-M (swap-AB stream-K) path.  Its split-K scratch
+// (partial tiles, per-tile arrival counters and a status word) lives in this file-scope device
+// array, so the entry point never allocates.  Every GPU that loads the library holds the array
+// until the process exits.  In host code `g_noalloc_scratch` is only a host-side stand-in for
+// the symbol: the device address is obtained with cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocPartialBytes = size_t(16) << 20;  // split-K partial tiles
+constexpr int kNoAllocCounters = 1 << 14;                  // n-tiles: N <= 2,097,152
+constexpr size_t kNoAllocBytes = kNoAllocPartialBytes + kNoAllocCounters * sizeof(int) + 256;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+
+struct NoAllocDevice {
+  bool ready = false;
+  int sms = 0;
+  unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoAllocDevice g_noalloc[kMaxDevices];
+
+fg_status noalloc_setup(int dev, NoAllocDevice** out) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  NoAllocDevice& d = g_noalloc[dev];
+  if (!d.ready) {
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return FG_ERR_CUDA;
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FG_ERR_CUDA;
+    if (major != 10) return FG_ERR_UNSUPPORTED;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FG_ERR_CUDA;
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FG_ERR_CUDA;
+    d.base = static_cast<unsigned char*>(ptr);
+    d.ready = true;
+  }
+  *out = &d;
+  return FG_OK;
+}
+
+template <int MP>
+fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* sfa, const void* B, const float* sfb,
+                           void* C, int M, int N, int K, cudaStream_t stream) {
+  constexpr int STAGES = swap_stages<MP>();
+  fg::SwapParams p;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.ws = reinterpret_cast<float*>(d.base);
+  p.counters = reinterpret_cast<int*>(d.base + kNoAllocPartialBytes);
+  p.status = p.counters + kNoAllocCounters;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.ld = fg_sfa_ld(M);
+  p.num_kb = (K + kBlockK - 1) / kBlockK;
+  p.n_tiles = (N + kBlockM - 1) / kBlockM;
+  if (p.n_tiles > kNoAllocCounters) return FG_ERR_UNSUPPORTED;
+  // the counters must start at zero; the kernel leaves them at zero, but a call that gave up a
+  // wait may not have, so clear the ones this call uses (a memset, no allocation)
+  if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.n_tiles) * sizeof(int), stream) != cudaSuccess)
+    return FG_ERR_CUDA;
+  CUtensorMap mW, mT;
+  if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
+  if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
+  // the partial tiles (two per CTA) must fit in the array: that caps the grid, not the problem size
+  const long long cap = static_cast<long long>(kNoAllocPartialBytes / (2 * MP * kBlockM * sizeof(float)));
+  long long grid = static_cast<long long>(p.n_tiles) * p.num_kb;
+  if (grid > d.sms) grid = d.sms;
+  if (grid > cap) grid = cap;
+  return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(static_cast<unsigned>(grid)),
+                                                               swap_smem_bytes<MP, STAGES>(), stream, mW, mT, &p);
+}
+
 }  // namespace
 
 extern "C" {
@@ -331,6 +408,37 @@ fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B
   if (!st) return s;
   return run_tiled<fg::kMasked>(st, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
                                 static_cast<cudaStream_t>(stream));
+}
+
+fg_status fp8_gemm_nt_noalloc(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M,
+                              int N, int K, void* stream) {
+  if (M < 0 || N < 0) return FG_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FG_OK;
+  fg_status s = check_common(A, sfa, B, sfb, C, N, K);
+  if (s != FG_OK) return s;
+  if (M > kMaxSwapMP) return FG_ERR_UNSUPPORTED;  // only the small-M kernel has this variant
+  if (static_cast<long long>(M) * K >= (1ll << 40) || static_cast<long long>(N) * K >= (1ll << 40))
+    return FG_ERR_UNSUPPORTED;
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return FG_ERR_CUDA;
+  NoAllocDevice* d = nullptr;
+  s = noalloc_setup(dev, &d);
+  if (s != FG_OK) return s;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (M <= 32) return run_swap_noalloc<32>(*d, A, sfa, B, sfb, C, M, N, K, cs);
+  if (M <= 64) return run_swap_noalloc<64>(*d, A, sfa, B, sfb, C, M, N, K, cs);
+  return run_swap_noalloc<128>(*d, A, sfa, B, sfb, C, M, N, K, cs);
+}
+
+fg_status fg_noalloc_status(void* stream) {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices || !g_noalloc[dev].ready) return FG_OK;  // never called here
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FG_ERR_CUDA;
+  int* status = reinterpret_cast<int*>(g_noalloc[dev].base + kNoAllocPartialBytes) + kNoAllocCounters;
+  int v = 0;
+  if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FG_ERR_CUDA;
+  if (v != 0 && cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
+  return static_cast<fg_status>(v);
 }
 
 fg_status fg_get_device_status(void* stream) {
