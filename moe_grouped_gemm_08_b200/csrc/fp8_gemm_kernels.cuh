@@ -48,7 +48,12 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, far above any legal wa
 constexpr int kErrTimeout = 6;       // FG_ERR_TIMEOUT
 constexpr int kMaskedMaxGroups = 1024;
 constexpr int kSwapScaleBytes = 24 * 1024;  // shared memory for staged combined scales (swap kernel)
-constexpr int kScaleChunk = 16;             // K blocks per staged scale chunk (tiled kernel)
+constexpr int kSaChunk = 8;                 // K blocks per staged scale chunk (tiled kernel)
+constexpr int kTiledThreads = 384;          // tiled kernel: three warpgroups
+constexpr int kTiledLaunchRegs = 168;       // registers per thread the tiled kernel is launched with
+constexpr int kPromoRegs = 232;             // after setmaxnreg: promotion warpgroups ...
+constexpr int kCtrlRegs = 40;               // ... and the producer / MMA warpgroup
+static_assert(2 * 128 * kPromoRegs + 128 * kCtrlRegs <= kTiledThreads * kTiledLaunchRegs, "register split");
 
 enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
@@ -157,62 +162,73 @@ __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* 
   return ti;
 }
 
-// Combined scales of one chunk of kScaleChunk K blocks of a 128-row tile,
-// s[kb][row] = sfa[kb][m0+row] * sfb[nb][kb], as held in registers by one
-// promotion thread (thread tid covers K block tid/16 and rows (tid%16)*8 .. +8).
+// Scales of one chunk of kSaChunk K blocks of a 128-row tile as held in registers by one
+// promotion thread: sfa for K block tid/32 and rows (tid%32)*4 .. +4, and (threads 0..15) one sfb
+// value for column half tid/kSaChunk and K block tid%kSaChunk.
 struct ScaleChunkRegs {
-  float v[8];
+  float4 a;
+  float b;
 };
 
 template <int MODE>
 __device__ __forceinline__ void load_scale_chunk(const TiledParams& p, const TileInfo& ti, int chunk, int tid,
-                                                 ScaleChunkRegs& r) {
-  const int kb = chunk * kScaleChunk + tid / 16;
-  const int r8 = (tid % 16) * 8;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) r.v[i] = 0.0f;
-  if (kb >= p.num_kb) return;
-  const int nb = ti.n0 / kBlockK;
-  const size_t g_sfb = (MODE == kDense) ? 0 : static_cast<size_t>(ti.g);
-  const float sb = __ldg(p.sfb + (g_sfb * p.num_nb + nb) * p.num_kb + kb);
-  const size_t g_sfa = (MODE == kMasked) ? static_cast<size_t>(ti.g) : 0;
-  const float* sa = p.sfa + (g_sfa * p.num_kb + kb) * static_cast<size_t>(p.ld) + ti.m0 + r8;
-  const int rows_left = p.M - (ti.m0 + r8);  // rows of the row space from this thread's first row on
-  if (rows_left >= 8) {
-    const float4 a0 = __ldg(reinterpret_cast<const float4*>(sa));
-    const float4 a1 = __ldg(reinterpret_cast<const float4*>(sa) + 1);
-    r.v[0] = a0.x * sb; r.v[1] = a0.y * sb; r.v[2] = a0.z * sb; r.v[3] = a0.w * sb;
-    r.v[4] = a1.x * sb; r.v[5] = a1.y * sb; r.v[6] = a1.z * sb; r.v[7] = a1.w * sb;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (i < rows_left) r.v[i] = __ldg(sa + i) * sb;
+                                                 int half_cols, ScaleChunkRegs& r) {
+  r.a = make_float4(0.f, 0.f, 0.f, 0.f);
+  r.b = 0.0f;
+  const int kb = chunk * kSaChunk + (tid >> 5);
+  const int r4 = (tid & 31) * 4;
+  if (kb < p.num_kb) {
+    const size_t g_sfa = (MODE == kMasked) ? static_cast<size_t>(ti.g) : 0;
+    const float* sa = p.sfa + (g_sfa * p.num_kb + kb) * static_cast<size_t>(p.ld) + ti.m0 + r4;
+    const int rows_left = p.M - (ti.m0 + r4);  // rows of the row space from this thread's first row on
+    if (rows_left >= 4) {
+      r.a = __ldg(reinterpret_cast<const float4*>(sa));
+    } else {
+      if (rows_left > 0) r.a.x = __ldg(sa);
+      if (rows_left > 1) r.a.y = __ldg(sa + 1);
+      if (rows_left > 2) r.a.z = __ldg(sa + 2);
+    }
+  }
+  if (tid < 2 * kSaChunk) {
+    const int h = tid / kSaChunk;
+    const int kb2 = chunk * kSaChunk + tid % kSaChunk;
+    const int nb = (ti.n0 + h * half_cols) / kBlockK;
+    if (kb2 < p.num_kb && nb < p.num_nb) {
+      const size_t g_sfb = (MODE == kDense) ? 0 : static_cast<size_t>(ti.g);
+      r.b = __ldg(p.sfb + (g_sfb * p.num_nb + nb) * p.num_kb + kb2);
+    }
   }
 }
 
+// chunk layout in shared memory: sa[kSaChunk][128] floats, then sb[2][kSaChunk] floats
 __device__ __forceinline__ void store_scale_chunk(float* buf, int tid, const ScaleChunkRegs& r) {
-  float4* dst = reinterpret_cast<float4*>(buf + (tid / 16) * kBlockM + (tid % 16) * 8);
-  dst[0] = make_float4(r.v[0], r.v[1], r.v[2], r.v[3]);
-  dst[1] = make_float4(r.v[4], r.v[5], r.v[6], r.v[7]);
+  reinterpret_cast<float4*>(buf + (tid >> 5) * kBlockM + (tid & 31) * 4)[0] = r.a;
+  if (tid < 2 * kSaChunk) buf[kSaChunk * kBlockM + tid] = r.b;
 }
 
-template <int BN, int STAGES, int NUM_TBUF, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+// Kernel 1 warp roles (384 threads, three warpgroups):
+//   warpgroup 0 (warps 0-3) and 1 (warps 4-7): promotion + epilogue, column halves 0 and 1; each
+//     raises its register budget to kPromoRegs so a thread can hold BN/2 fp32 accumulators;
+//   warpgroup 2: warp 8 TMA producer, warp 9 TMEM owner + MMA issuer, warps 10-11 idle; it lowers
+//     its budget to kCtrlRegs.  The split assumes the kernel is launched with kTiledLaunchRegs
+//     registers per thread, which the host checks before every launch.
+template <int BN, int STAGES, int MODE>
+__global__ void __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const TiledParams p) {
-  static_assert(BN == 128, "one 128-wide block of B scales per tile");
+  static_assert(BN == 128 || BN == 256, "BN");
   constexpr int A_BYTES = kBlockM * kBlockK;
   constexpr int B_BYTES = BN * kBlockK;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int NUM_TBUF = 512 / BN;
   constexpr uint32_t TMEM_COLS = NUM_TBUF * BN;
-  static_assert(TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   constexpr int COLS = BN / 2;  // columns per promotion thread
-  constexpr int CHUNK_FLOATS = kScaleChunk * kBlockM;
+  constexpr int CHUNK_FLOATS = kSaChunk * kBlockM + 2 * kSaChunk;
   constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, BN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
-  float* s_scale = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [2][kScaleChunk][128]
+  float* s_scale = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [2][CHUNK_FLOATS]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + 2 * CHUNK_FLOATS);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -226,23 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Producer state (lane 0 of the producer warp): tile walk position, smem ring position, loads issued.
-  int p_t = blockIdx.x, p_kb = 0;
-  TileInfo p_ti;
-  p_ti.live = 0;
-  uint32_t p_stage = 0, p_phase = 0;
-  uint64_t p_issued = 0;
-  const bool producer = (warp == kProducerWarp && lane == 0);
-  auto issue = [&](const TileInfo& ti, int kb) {
-    uint8_t* sa = smem + p_stage * STAGE_BYTES;
-    mbar_arrive_expect_tx(&full[p_stage], STAGE_BYTES);
-    tma_load_3d(sa, &tmA, &full[p_stage], kb * kBlockK, ti.m0, (MODE == kMasked) ? ti.g : 0);
-    tma_load_3d(sa + A_BYTES, &tmB, &full[p_stage], kb * kBlockK, ti.n0, (MODE == kDense) ? 0 : ti.g);
-    ++p_issued;
-    if (++p_stage == STAGES) { p_stage = 0; p_phase ^= 1u; }
-  };
-
-  if (producer) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -294,32 +294,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     num_tiles = p.m_blocks * p.n_blocks;
   }
 
-  if (warp == kProducerWarp) {
-    if (lane == 0) {
+  if (warp >= kPromoWarps) {
+    // ================================================ warpgroup 2: producer, MMA, idle warps
+    reg_dealloc<kCtrlRegs>();
+    if (warp == kProducerWarp && lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0;
       bool ok = true;
-      for (; p_t < num_tiles; p_t += gridDim.x) {  // this CTA's first live tile
-        p_ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, p_t, BN);
-        if (p_ti.live) break;
-      }
-      while (p_t < num_tiles) {
-        if (!mbar_wait(&empty[p_stage], p_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-        issue(p_ti, p_kb);
-        if (++p_kb == p.num_kb) {
-          p_kb = 0;
-          for (p_t += gridDim.x; p_t < num_tiles; p_t += gridDim.x) {
-            p_ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, p_t, BN);
-            if (p_ti.live) break;
-          }
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+        if (!ti.live) continue;
+        const int ga = (MODE == kMasked) ? ti.g : 0;
+        const int gb = (MODE == kDense) ? 0 : ti.g;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          uint8_t* st = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+          tma_load_3d(st, &tmA, &full[stage], kb * kBlockK, ti.m0, ga);
+          tma_load_3d(st + A_BYTES, &tmB, &full[stage], kb * kBlockK, ti.n0, gb);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
       }
       if (!ok) {  // drain this CTA's copies still in flight before the CTA exits
-        const uint64_t first = p_issued > STAGES ? p_issued - STAGES : 0;
-        for (uint64_t i = first; i < p_issued; ++i)
-          mbar_drain(&full[i % STAGES], static_cast<uint32_t>((i / STAGES) & 1));
+        const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+        for (uint32_t i = first; i < issued; ++i) mbar_drain(&full[i % STAGES], (i / STAGES) & 1u);
       }
-    }
-  } else if (warp == kMmaWarp) {
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
       uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
@@ -330,9 +331,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem_base + tb * BN;
-          const uint32_t sa = smem_addr(smem + stage * STAGE_BYTES);
-          const uint64_t adesc = smem_desc_k128_sw128(sa);
-          const uint64_t bdesc = smem_desc_k128_sw128(sa + A_BYTES);
+          const uint32_t st = smem_addr(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = smem_desc_k128_sw128(st);
+          const uint64_t bdesc = smem_desc_k128_sw128(st + A_BYTES);
 #pragma unroll
           for (int j = 0; j < kBlockK / 32; ++j)  // 32 e4m3 = 32 bytes = 2 descriptor units per step
             mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
@@ -347,13 +348,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_drain(mma_done, 0);
     }
   } else {
-    // ------------------------------------------------ promotion + epilogue
+    // ================================================ warpgroups 0-1: promotion + epilogue
+    reg_alloc<kPromoRegs>();
     const int q = warp & 3;
     const int h = warp >> 2;
     const int row = q * 32 + lane;
     const int tid = threadIdx.x;  // 0..255 among promotion threads
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int n_chunks = (p.num_kb + kScaleChunk - 1) / kScaleChunk;
+    const int n_chunks = (p.num_kb + kSaChunk - 1) / kSaChunk;
     uint32_t tb = 0, tphase = 0, pphase = 0;
     bool ok = true;
 
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ScaleChunkRegs nxt;
     int buf = 0;
     if (t < num_tiles) {
-      load_scale_chunk<MODE>(p, ti, 0, tid, nxt);
+      load_scale_chunk<MODE>(p, ti, 0, tid, COLS, nxt);
       store_scale_chunk(s_scale, tid, nxt);
       ok = group_sync(pbar, pphase, abort_flag);
     }
@@ -393,26 +395,33 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       for (int c = 0; c < n_chunks && ok; ++c) {
         // prefetch the next chunk of the sequence into registers
-        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, nxt);
-        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, nxt);
-        const float* sc = s_scale + buf * CHUNK_FLOATS + row;
-        const int kb_end = (c + 1) * kScaleChunk < p.num_kb ? (c + 1) * kScaleChunk : p.num_kb;
-        for (int kb = c * kScaleChunk; kb < kb_end; ++kb) {
-          const float s = sc[(kb - c * kScaleChunk) * kBlockM];
+        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, COLS, nxt);
+        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, COLS, nxt);
+        const float* sa = s_scale + buf * CHUNK_FLOATS + row;
+        const float* sb = s_scale + buf * CHUNK_FLOATS + kSaChunk * kBlockM + h * kSaChunk;
+        const int kb_end = (c + 1) * kSaChunk < p.num_kb ? (c + 1) * kSaChunk : p.num_kb;
+        for (int kb = c * kSaChunk; kb < kb_end; ++kb) {
+          const int kl = kb - c * kSaChunk;
+          const float s = sa[kl * kBlockM] * sb[kl];
           if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
-          uint32_t v0[32], v1[32];
-          tmem_ld_32x32b_x32(taddr, v0);
-          tmem_ld_32x32b_x32(taddr + 32, v1);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[tb]);  // hand the TMEM buffer back to the MMA
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            acc[j] = fmaf(__uint_as_float(v0[j]), s, acc[j]);
-            acc[32 + j] = fmaf(__uint_as_float(v1[j]), s, acc[32 + j]);
+          for (int c0 = 0; c0 < COLS; c0 += 64) {
+            uint32_t v0[32], v1[32];
+            tmem_ld_32x32b_x32(taddr + c0, v0);
+            tmem_ld_32x32b_x32(taddr + c0 + 32, v1);
+            tmem_wait_ld();
+            if (c0 + 64 >= COLS) {  // whole slice read: hand the TMEM buffer back to the MMA
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tempty[tb]);
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              acc[c0 + j] = fmaf(__uint_as_float(v0[j]), s, acc[c0 + j]);
+              acc[c0 + 32 + j] = fmaf(__uint_as_float(v1[j]), s, acc[c0 + 32 + j]);
+            }
           }
           if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }

@@ -40,15 +40,14 @@ EncodeTiledFn g_encode = nullptr;
 std::atomic<int> g_dense_path{0};
 std::atomic<uint64_t> g_launches{0};
 
-// tiled kernel configuration
-constexpr int kTiledBN = 128;
-constexpr int kTiledStages = 6;
-constexpr int kTiledTbuf = 4;
+// tiled kernel configuration: 128 x 256 output tiles, 4-stage ring
+constexpr int kTiledBN = 256;
+constexpr int kTiledStages = 4;
 
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBlockM + BN) * kBlockK +
-         2 * fg::kScaleChunk * kBlockM * 4 /*scale chunks*/ + 256 /*barriers*/ +
+         2 * (fg::kSaChunk * kBlockM + 2 * fg::kSaChunk) * 4 /*scale chunks*/ + 256 /*barriers*/ +
          4 * (fg::kMaskedMaxGroups + 1) /*masked prefix*/;
 }
 
@@ -106,9 +105,12 @@ bool encode_fp8_map_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t 
 }
 
 // One instantiation per kernel, so the once-per-device flag below is per kernel.
+// threads: block size.  required_regs > 0: the kernel re-splits its registers between warpgroups
+// (setmaxnreg) assuming exactly that many registers per thread at launch; refuse to launch a
+// build where the compiler chose another count (the split would never be granted).
 template <auto KERNEL>
 fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap& m0, const CUtensorMap& m1,
-                 const void* params_ptr) {
+                 const void* params_ptr, int threads = fg::kThreads, int required_regs = 0) {
   // the opt-in shared-memory size is a per-function attribute: set once per device (so that a
   // call made during stream capture issues no attribute change)
   const auto kernel = KERNEL;
@@ -116,6 +118,11 @@ fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap&
   const int dev = current_device();
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load(std::memory_order_acquire) & bit)) {
+    if (required_regs > 0) {
+      cudaFuncAttributes fa;
+      if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return FG_ERR_CUDA;
+      if (fa.numRegs != required_regs) return FG_ERR_UNSUPPORTED;
+    }
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
         cudaSuccess)
       return FG_ERR_CUDA;
@@ -131,7 +138,7 @@ fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap&
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(fg::kThreads, 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
@@ -183,8 +190,8 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
 
   long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
   const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
-  return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, kTiledTbuf, MODE>>(
-      dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, mA, mB, &p);
+  return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, MODE>>(dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, mA,
+                                                              mB, &p, fg::kTiledThreads, fg::kTiledLaunchRegs);
 }
 
 template <int MP>
