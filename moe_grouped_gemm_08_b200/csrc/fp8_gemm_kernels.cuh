@@ -164,7 +164,8 @@ __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* 
 
 // Scales of one chunk of kSaChunk K blocks of a 128-row tile as held in registers by one
 // promotion thread: sfa for K block tid/32 and rows (tid%32)*4 .. +4, and (threads 0..15) one sfb
-// value for column half tid/kSaChunk and K block tid%kSaChunk.
+// value: 128-column block nb0 + tid/kSaChunk of the tile (a tile spans at most two), K block
+// tid%kSaChunk.
 struct ScaleChunkRegs {
   float4 a;
   float b;
@@ -172,7 +173,7 @@ struct ScaleChunkRegs {
 
 template <int MODE>
 __device__ __forceinline__ void load_scale_chunk(const TiledParams& p, const TileInfo& ti, int chunk, int tid,
-                                                 int half_cols, ScaleChunkRegs& r) {
+                                                 ScaleChunkRegs& r) {
   r.a = make_float4(0.f, 0.f, 0.f, 0.f);
   r.b = 0.0f;
   const int kb = chunk * kSaChunk + (tid >> 5);
@@ -190,9 +191,8 @@ __device__ __forceinline__ void load_scale_chunk(const TiledParams& p, const Til
     }
   }
   if (tid < 2 * kSaChunk) {
-    const int h = tid / kSaChunk;
     const int kb2 = chunk * kSaChunk + tid % kSaChunk;
-    const int nb = (ti.n0 + h * half_cols) / kBlockK;
+    const int nb = ti.n0 / kBlockK + tid / kSaChunk;
     if (kb2 < p.num_kb && nb < p.num_nb) {
       const size_t g_sfb = (MODE == kDense) ? 0 : static_cast<size_t>(ti.g);
       r.b = __ldg(p.sfb + (g_sfb * p.num_nb + nb) * p.num_kb + kb2);
@@ -206,29 +206,42 @@ __device__ __forceinline__ void store_scale_chunk(float* buf, int tid, const Sca
   if (tid < 2 * kSaChunk) buf[kSaChunk * kBlockM + tid] = r.b;
 }
 
+// Output staging of one promotion warp: its 32 rows x COLS columns as COLS/32 boxes of 32 x 32
+// bf16 (64-byte rows, 64-byte swizzle: the 16-byte chunk c of row r sits at chunk c ^ ((r/2)%4)),
+// the layout the C tensor map stores from.
+constexpr int kStoreBoxBytes = 32 * 64;
+
 // Kernel 1 warp roles (384 threads, three warpgroups):
 //   warpgroup 0 (warps 0-3) and 1 (warps 4-7): promotion + epilogue, column halves 0 and 1; each
-//     raises its register budget to kPromoRegs so a thread can hold BN/2 fp32 accumulators;
+//     raises its register budget to kPromoRegs so a thread can hold the BN/2 fp32 accumulators of
+//     its row and one whole BN/2-column slice loaded from TMEM;
 //   warpgroup 2: warp 8 TMA producer, warp 9 TMEM owner + MMA issuer, warps 10-11 idle; it lowers
 //     its budget to kCtrlRegs.  The split assumes the kernel is launched with kTiledLaunchRegs
 //     registers per thread, which the host checks before every launch.
+// BN = 192 keeps one slice read (three 32-column TMEM loads) per K block within the register
+// budget, so each TMEM buffer is handed back after a single load round trip; two buffers of 192
+// columns fit the 512 TMEM columns.
 template <int BN, int STAGES, int MODE>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const TiledParams p) {
-  static_assert(BN == 128 || BN == 256, "BN");
+                          const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
+  constexpr int COLS = BN / 2;  // columns per promotion thread
+  constexpr int NCH = COLS / 32;  // 32-column TMEM loads (and store boxes) per thread
+  // tiles start at multiples of 64 columns, so no 32-column chunk straddles a 128-column sfb block
+  static_assert(COLS % 32 == 0 && BN <= 256, "BN");
   constexpr int A_BYTES = kBlockM * kBlockK;
   constexpr int B_BYTES = BN * kBlockK;
   constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr int NUM_TBUF = 512 / BN;
-  constexpr uint32_t TMEM_COLS = NUM_TBUF * BN;
-  constexpr int COLS = BN / 2;  // columns per promotion thread
+  constexpr uint32_t TMEM_COLS = 512;
   constexpr int CHUNK_FLOATS = kSaChunk * kBlockM + 2 * kSaChunk;
   constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, BN);
+  constexpr int WARP_STORE_BYTES = NCH * kStoreBoxBytes;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
-  float* s_scale = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);  // [2][CHUNK_FLOATS]
+  uint8_t* s_out = smem + STAGES * STAGE_BYTES;                                    // [8 warps][NCH boxes]
+  float* s_scale = reinterpret_cast<float*>(s_out + kPromoWarps * WARP_STORE_BYTES);  // [2][CHUNK_FLOATS]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + 2 * CHUNK_FLOATS);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -245,6 +258,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
     mbar_init(mma_done, 1);
@@ -356,6 +370,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const int tid = threadIdx.x;  // 0..255 among promotion threads
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int n_chunks = (p.num_kb + kSaChunk - 1) / kSaChunk;
+    uint8_t* s_w = s_out + warp * WARP_STORE_BYTES;  // this warp's output staging
+    bool stores_pending = false;
     uint32_t tb = 0, tphase = 0, pphase = 0;
     bool ok = true;
 
@@ -374,7 +390,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     ScaleChunkRegs nxt;
     int buf = 0;
     if (t < num_tiles) {
-      load_scale_chunk<MODE>(p, ti, 0, tid, COLS, nxt);
+      load_scale_chunk<MODE>(p, ti, 0, tid, nxt);
       store_scale_chunk(s_scale, tid, nxt);
       ok = group_sync(pbar, pphase, abort_flag);
     }
@@ -388,6 +404,11 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         if (ti_next.live) break;
       }
       const int m = ti.m0 + row;
+      // sfb block (0: the tile's first, 1: the next) of each 32-column chunk of this thread
+      uint32_t hi_mask = 0;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+        hi_mask |= static_cast<uint32_t>((ti.n0 + h * COLS + 32 * i) / kBlockK - ti.n0 / kBlockK) << i;
 
       float acc[COLS];
 #pragma unroll
@@ -395,33 +416,33 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 
       for (int c = 0; c < n_chunks && ok; ++c) {
         // prefetch the next chunk of the sequence into registers
-        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, COLS, nxt);
-        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, COLS, nxt);
+        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, nxt);
+        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, nxt);
         const float* sa = s_scale + buf * CHUNK_FLOATS + row;
-        const float* sb = s_scale + buf * CHUNK_FLOATS + kSaChunk * kBlockM + h * kSaChunk;
+        const float* sb = s_scale + buf * CHUNK_FLOATS + kSaChunk * kBlockM;
         const int kb_end = (c + 1) * kSaChunk < p.num_kb ? (c + 1) * kSaChunk : p.num_kb;
         for (int kb = c * kSaChunk; kb < kb_end; ++kb) {
           const int kl = kb - c * kSaChunk;
-          const float s = sa[kl * kBlockM] * sb[kl];
+          const float sav = sa[kl * kBlockM];
+          const float s0 = sav * sb[kl];
+          const float s1 = sav * sb[kSaChunk + kl];
           if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
+          uint32_t v[NCH][32];
 #pragma unroll
-          for (int c0 = 0; c0 < COLS; c0 += 64) {
-            uint32_t v0[32], v1[32];
-            tmem_ld_32x32b_x32(taddr + c0, v0);
-            tmem_ld_32x32b_x32(taddr + c0 + 32, v1);
-            tmem_wait_ld();
-            if (c0 + 64 >= COLS) {  // whole slice read: hand the TMEM buffer back to the MMA
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&tempty[tb]);
-            }
+          for (int i = 0; i < NCH; ++i) tmem_ld_32x32b_x32(taddr + 32 * i, v[i]);
+          tmem_wait_ld();
+          // whole slice read: hand the TMEM buffer back to the MMA
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              acc[c0 + j] = fmaf(__uint_as_float(v0[j]), s, acc[c0 + j]);
-              acc[c0 + 32 + j] = fmaf(__uint_as_float(v1[j]), s, acc[c0 + 32 + j]);
-            }
+          for (int i = 0; i < NCH; ++i) {
+            const float s = ((hi_mask >> i) & 1u) ? s1 : s0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+              ffma2(acc[32 * i + j], acc[32 * i + j + 1], __uint_as_float(v[i][j]), __uint_as_float(v[i][j + 1]), s);
           }
           if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }
@@ -434,35 +455,71 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       }
       if (!ok) break;
 
-      // epilogue: bf16 round-to-nearest-even, 16-byte stores of this thread's row segment
+      // epilogue: bf16 round-to-nearest-even.  A warp whose 32 rows are all to be written stages
+      // them in shared memory and stores them with TMA; a warp with rows that must stay untouched
+      // (past M, past masked_m, padding rows of another group) stores its valid rows directly.
       bool store_row = m < p.M;
-      __nv_bfloat16* crow;
+      int cnt = p.M;
       if (MODE == kMasked) {
-        int cnt = __ldg(p.masked_m + ti.g);
+        cnt = __ldg(p.masked_m + ti.g);
         cnt = cnt > p.M ? p.M : cnt;
         store_row = m < cnt;
-        crow = p.C + (static_cast<size_t>(ti.g) * p.M + m) * p.N;
-      } else {
-        if (MODE == kContiguous && store_row) store_row = __ldg(p.m_indices + m) == ti.g;
-        crow = p.C + static_cast<size_t>(m) * p.N;
+      } else if (MODE == kContiguous) {
+        if (store_row) store_row = __ldg(p.m_indices + m) == ti.g;
       }
-      if (store_row) {
-        const int nbase = ti.n0 + h * COLS;
+      const int nbase = ti.n0 + h * COLS;
+      if (__all_sync(0xffffffffu, store_row)) {
+        if (stores_pending) {  // the previous tile's stores must have read the staging area
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+        }
+        const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          uint8_t* box_row = s_w + i * kStoreBoxBytes + lane * 64;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint4 val;
+            val.x = pack_bf16x2(acc[32 * i + 8 * c + 0], acc[32 * i + 8 * c + 1]);
+            val.y = pack_bf16x2(acc[32 * i + 8 * c + 2], acc[32 * i + 8 * c + 3]);
+            val.z = pack_bf16x2(acc[32 * i + 8 * c + 4], acc[32 * i + 8 * c + 5]);
+            val.w = pack_bf16x2(acc[32 * i + 8 * c + 6], acc[32 * i + 8 * c + 7]);
+            *reinterpret_cast<uint4*>(box_row + ((c ^ sw) << 4)) = val;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = ti.m0 + q * 32;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            if (nbase + 32 * i < p.N) {
+              if (MODE == kMasked) tma_store_3d(&tmC, s_w + i * kStoreBoxBytes, nbase + 32 * i, y, ti.g);
+              else tma_store_2d(&tmC, s_w + i * kStoreBoxBytes, nbase + 32 * i, y);
+            }
+          }
+          bulk_commit_group();
+        }
+        stores_pending = true;
+      } else if (store_row) {
+        __nv_bfloat16* crow = (MODE == kMasked) ? p.C + (static_cast<size_t>(ti.g) * p.M + m) * p.N
+                                                : p.C + static_cast<size_t>(m) * p.N;
 #pragma unroll
         for (int j = 0; j < COLS; j += 8) {
           if (nbase + j < p.N) {
-            uint4 v;
-            v.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
-            v.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-            v.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-            v.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
-            *reinterpret_cast<uint4*>(crow + nbase + j) = v;
+            uint4 val;
+            val.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
+            val.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
+            val.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
+            val.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+            *reinterpret_cast<uint4*>(crow + nbase + j) = val;
           }
         }
       }
       t = t_next;
       ti = ti_next;
     }
+    if (stores_pending && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

@@ -40,16 +40,18 @@ EncodeTiledFn g_encode = nullptr;
 std::atomic<int> g_dense_path{0};
 std::atomic<uint64_t> g_launches{0};
 
-// tiled kernel configuration: 128 x 256 output tiles, 4-stage ring
-constexpr int kTiledBN = 256;
+// tiled kernel configuration: 128 x 192 output tiles, 4-stage ring
+constexpr int kTiledBN = 192;
 constexpr int kTiledStages = 4;
 
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBlockM + BN) * kBlockK +
+         static_cast<size_t>(fg::kPromoWarps) * (BN / 64) * fg::kStoreBoxBytes /*output staging*/ +
          2 * (fg::kSaChunk * kBlockM + 2 * fg::kSaChunk) * 4 /*scale chunks*/ + 256 /*barriers*/ +
          4 * (fg::kMaskedMaxGroups + 1) /*masked prefix*/;
 }
+static_assert(tiled_smem_bytes<kTiledBN, kTiledStages>() <= 227 * 1024, "tiled kernel shared memory");
 
 template <int MP>
 constexpr int swap_stages() {
@@ -93,6 +95,19 @@ bool encode_fp8_map(CUtensorMap* map, const void* base, uint64_t K, uint64_t row
   return r == CUDA_SUCCESS;
 }
 
+// bf16 output map for TMA stores: dims {N, rows[, groups]}, box {32, 32[, 1]}, 64-byte swizzle
+// (the staging layout of the tiled kernel's epilogue).
+bool encode_bf16_store_map(CUtensorMap* map, void* base, uint64_t N, uint64_t rows, uint64_t groups, bool three_d) {
+  cuuint64_t dims[3] = {N, rows, groups};
+  cuuint64_t strides[2] = {N * 2, N * 2 * rows};
+  cuuint32_t box[3] = {32, 32, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, three_d ? 3 : 2, base, dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_fp8_map_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
   cuuint64_t dims[2] = {K, rows};
   cuuint64_t strides[1] = {K};
@@ -108,9 +123,9 @@ bool encode_fp8_map_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t 
 // threads: block size.  required_regs > 0: the kernel re-splits its registers between warpgroups
 // (setmaxnreg) assuming exactly that many registers per thread at launch; refuse to launch a
 // build where the compiler chose another count (the split would never be granted).
+// args: pointers to the kernel's arguments, in order.
 template <auto KERNEL>
-fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap& m0, const CUtensorMap& m1,
-                 const void* params_ptr, int threads = fg::kThreads, int required_regs = 0) {
+fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, void** args, int threads, int required_regs = 0) {
   // the opt-in shared-memory size is a per-function attribute: set once per device (so that a
   // call made during stream capture issues no attribute change)
   const auto kernel = KERNEL;
@@ -128,7 +143,6 @@ fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, const CUtensorMap&
       return FG_ERR_CUDA;
     configured.fetch_or(bit, std::memory_order_acq_rel);
   }
-  void* args[3] = {const_cast<CUtensorMap*>(&m0), const_cast<CUtensorMap*>(&m1), const_cast<void*>(params_ptr)};
   // programmatic dependent launch: the kernel's prologue (barriers, TMEM allocation, descriptor
   // prefetch) may overlap the previous kernel of the stream; the kernel waits for that kernel
   // (griddepcontrol.wait) before its first global-memory access
@@ -182,16 +196,18 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
   p.m_blocks = (M + kBlockM - 1) / kBlockM;
   p.n_blocks = (N + BN - 1) / BN;
 
-  CUtensorMap mA, mB;
+  CUtensorMap mA, mB, mC;
   const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;
   const uint64_t groupsB = (MODE == fg::kDense) ? 1 : static_cast<uint64_t>(G);
   if (!encode_fp8_map(&mA, A, K, M, groupsA, kBlockM)) return FG_ERR_CUDA;
   if (!encode_fp8_map(&mB, B, K, N, groupsB, BN)) return FG_ERR_CUDA;
+  if (!encode_bf16_store_map(&mC, C, N, M, groupsA, MODE == fg::kMasked)) return FG_ERR_CUDA;
 
   long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
   const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
-  return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, MODE>>(dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, mA,
-                                                              mB, &p, fg::kTiledThreads, fg::kTiledLaunchRegs);
+  void* args[4] = {&mA, &mB, &mC, &p};
+  return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, MODE>>(dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, args,
+                                                              fg::kTiledThreads, fg::kTiledLaunchRegs);
 }
 
 template <int MP>
@@ -218,8 +234,9 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
   if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
   const long long units = static_cast<long long>(p.n_tiles) * p.num_kb;
   const int grid = static_cast<int>(units < st->sms ? units : st->sms);
+  void* args[3] = {&mW, &mT, &p};
   return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(grid), swap_smem_bytes<MP, STAGES>(), stream,
-                                                               mW, mT, &p);
+                                                               args, fg::kThreads);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -295,8 +312,10 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   long long grid = static_cast<long long>(p.n_tiles) * p.num_kb;
   if (grid > d.sms) grid = d.sms;
   if (grid > cap) grid = cap;
+  void* args[3] = {&mW, &mT, &p};
   return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(static_cast<unsigned>(grid)),
-                                                               swap_smem_bytes<MP, STAGES>(), stream, mW, mT, &p);
+                                                               swap_smem_bytes<MP, STAGES>(), stream, args,
+                                                               fg::kThreads);
 }
 
 }  // namespace
