@@ -76,6 +76,37 @@ def load_traffic(kernel: str, workload: str):
     return entry
 
 
+def record_traffic(csv_path: str, workload: str) -> None:
+    """Average dram__bytes_read.sum + dram__bytes_write.sum per launch of each of this library's
+    kernels in an ncu --csv launch list, stored in profiles/traffic.json with the kernel source hash."""
+    import csv as _csv
+    rows = [r for r in _csv.reader(open(csv_path)) if r]
+    hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r and "Metric Name" in r)
+    h = rows[hi]
+    col = {k: h.index(k) for k in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    per = {}
+    for r in rows[hi + 1:]:
+        if len(r) != len(h) or not r[col["Metric Name"]].startswith("dram__bytes_"):
+            continue
+        name = r[col["Kernel Name"]]
+        kern = next((k for k in ("fp8_gemm_swap_streamk_kernel", "fp8_gemm_tiled_kernel") if k in name), None)
+        if kern is None:
+            continue
+        v = float(r[col["Metric Value"]].replace(",", "")) * scale.get(r[col["Metric Unit"]], 1)
+        per.setdefault(kern, {}).setdefault(r[col["ID"]], 0.0)
+        per[kern][r[col["ID"]]] += v
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    d = json.load(open(path)) if os.path.exists(path) else {}
+    for kern, launches in per.items():
+        d[f"{kern}:{workload}"] = {"dram_bytes_per_launch": round(sum(launches.values()) / len(launches)),
+                                   "launches": len(launches), "kernel_source_hash": kernel_source_hash(),
+                                   "source": os.path.basename(csv_path)}
+    with open(path, "w") as f:
+        json.dump(d, f, indent=1, sort_keys=True)
+    print(json.dumps({k: v for k, v in d.items() if k.endswith(":" + workload)}))
+
+
 def cdiv(a, b):
     return (a + b - 1) // b
 
@@ -523,7 +554,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--record-traffic", default=None, metavar="CSV",
+                    help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()
+    if args.record_traffic:
+        record_traffic(args.record_traffic, workload_list(args.workload, args.shape)[0])
+        return
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = dist_setup(args)

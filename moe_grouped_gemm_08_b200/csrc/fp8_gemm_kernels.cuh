@@ -73,6 +73,7 @@ struct TiledParams {
   int num_nb;   // ceil(N / 128): sfb blocks per group
   int m_blocks; // ceil(M / 128)
   int n_blocks; // ceil(N / BN)
+  int group_m;  // tile order: groups of group_m m-blocks, m-block fastest inside a group
 };
 
 struct SwapParams {
@@ -129,13 +130,26 @@ struct TileInfo {
   int n0;
 };
 
+// Tile t of the walk -> (m-block, n-block).  The m-blocks (masked: the live ones) form groups of
+// group_m; a group's tiles are consecutive, m-block fastest, so while a group is being worked on
+// its A rows are re-read from L2 by every n-block rather than from DRAM.
+__device__ __forceinline__ void tile_coords(int t, int mblocks, int n_blocks, int group_m, int& mb, int& nb) {
+  const int per_group = group_m * n_blocks;
+  const int mg = t / per_group;
+  const int rem = t - mg * per_group;
+  const int gm0 = mg * group_m;
+  const int gm = (mblocks - gm0) < group_m ? (mblocks - gm0) : group_m;
+  nb = rem / gm;
+  mb = gm0 + (rem - nb * gm);
+}
+
 template <int MODE>
 __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* s_prefix, int live_mblocks, int t,
                                                int BN) {
   TileInfo ti;
   if (MODE == kMasked) {
-    const int nb = t / live_mblocks;
-    const int lm = t - nb * live_mblocks;
+    int lm, nb;
+    tile_coords(t, live_mblocks, p.n_blocks, p.group_m, lm, nb);
     int lo = 0, hi = p.G;  // largest g with s_prefix[g] <= lm
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
@@ -146,8 +160,8 @@ __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* 
     ti.m0 = (lm - s_prefix[lo]) * kBlockM;
     ti.n0 = nb * BN;
   } else {
-    const int nb = t / p.m_blocks;
-    const int mb = t - nb * p.m_blocks;
+    int mb, nb;
+    tile_coords(t, p.m_blocks, p.n_blocks, p.group_m, mb, nb);
     ti.m0 = mb * kBlockM;
     ti.n0 = nb * BN;
     if (MODE == kContiguous) {
@@ -315,6 +329,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0;
       bool ok = true;
+      const uint64_t pol_a = l2_policy_evict_last();   // A rows: re-read by every n-block of a group
+      const uint64_t pol_b = l2_policy_evict_first();  // B tiles: shared by the concurrent m-blocks only
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
         if (!ti.live) continue;
@@ -324,8 +340,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           uint8_t* st = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          tma_load_3d(st, &tmA, &full[stage], kb * kBlockK, ti.m0, ga);
-          tma_load_3d(st + A_BYTES, &tmB, &full[stage], kb * kBlockK, ti.n0, gb);
+          tma_load_3d(st, &tmA, &full[stage], kb * kBlockK, ti.m0, ga, pol_a);
+          tma_load_3d(st + A_BYTES, &tmB, &full[stage], kb * kBlockK, ti.n0, gb, pol_b);
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -410,9 +426,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       for (int i = 0; i < NCH; ++i)
         hi_mask |= static_cast<uint32_t>((ti.n0 + h * COLS + 32 * i) / kBlockK - ti.n0 / kBlockK) << i;
 
-      float acc[COLS];
+      float2 acc[COLS / 2];  // column pairs: promoted with the packed fp32 FMA
 #pragma unroll
-      for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
       for (int c = 0; c < n_chunks && ok; ++c) {
         // prefetch the next chunk of the sequence into registers
@@ -440,9 +456,11 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
           for (int i = 0; i < NCH; ++i) {
             const float s = ((hi_mask >> i) & 1u) ? s1 : s0;
+            const float2 s2 = make_float2(s, s);
 #pragma unroll
-            for (int j = 0; j < 32; j += 2)
-              ffma2(acc[32 * i + j], acc[32 * i + j + 1], __uint_as_float(v[i][j]), __uint_as_float(v[i][j + 1]), s);
+            for (int j = 0; j < 16; ++j)
+              acc[16 * i + j] = __ffma2_rn(make_float2(__uint_as_float(v[i][2 * j]), __uint_as_float(v[i][2 * j + 1])),
+                                           s2, acc[16 * i + j]);
           }
           if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }
@@ -479,11 +497,12 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           uint8_t* box_row = s_w + i * kStoreBoxBytes + lane * 64;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
+            const float2* a = acc + 16 * i + 4 * c;
             uint4 val;
-            val.x = pack_bf16x2(acc[32 * i + 8 * c + 0], acc[32 * i + 8 * c + 1]);
-            val.y = pack_bf16x2(acc[32 * i + 8 * c + 2], acc[32 * i + 8 * c + 3]);
-            val.z = pack_bf16x2(acc[32 * i + 8 * c + 4], acc[32 * i + 8 * c + 5]);
-            val.w = pack_bf16x2(acc[32 * i + 8 * c + 6], acc[32 * i + 8 * c + 7]);
+            val.x = pack_bf16x2(a[0].x, a[0].y);
+            val.y = pack_bf16x2(a[1].x, a[1].y);
+            val.z = pack_bf16x2(a[2].x, a[2].y);
+            val.w = pack_bf16x2(a[3].x, a[3].y);
             *reinterpret_cast<uint4*>(box_row + ((c ^ sw) << 4)) = val;
           }
         }
@@ -507,11 +526,12 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
         for (int j = 0; j < COLS; j += 8) {
           if (nbase + j < p.N) {
+            const float2* a = acc + j / 2;
             uint4 val;
-            val.x = pack_bf16x2(acc[j + 0], acc[j + 1]);
-            val.y = pack_bf16x2(acc[j + 2], acc[j + 3]);
-            val.z = pack_bf16x2(acc[j + 4], acc[j + 5]);
-            val.w = pack_bf16x2(acc[j + 6], acc[j + 7]);
+            val.x = pack_bf16x2(a[0].x, a[0].y);
+            val.y = pack_bf16x2(a[1].x, a[1].y);
+            val.z = pack_bf16x2(a[2].x, a[2].y);
+            val.w = pack_bf16x2(a[3].x, a[3].y);
             *reinterpret_cast<uint4*>(crow + nbase + j) = val;
           }
         }

@@ -40,9 +40,15 @@ EncodeTiledFn g_encode = nullptr;
 std::atomic<int> g_dense_path{0};
 std::atomic<uint64_t> g_launches{0};
 
-// tiled kernel configuration: 128 x 192 output tiles, 4-stage ring
-constexpr int kTiledBN = 192;
-constexpr int kTiledStages = 4;
+// tiled kernel configuration: 128 x 192 output tiles, 4-stage ring (overridable when building)
+#ifndef FG_TILED_BN
+#define FG_TILED_BN 192
+#endif
+#ifndef FG_TILED_STAGES
+#define FG_TILED_STAGES 4
+#endif
+constexpr int kTiledBN = FG_TILED_BN;
+constexpr int kTiledStages = FG_TILED_STAGES;
 
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
@@ -195,6 +201,16 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
   p.num_nb = (N + kBlockK - 1) / kBlockK;
   p.m_blocks = (M + kBlockM - 1) / kBlockM;
   p.n_blocks = (N + BN - 1) / BN;
+  // m-blocks per group of the tile walk: a group's A rows (128 * K bytes per m-block) should stay
+  // in L2 (126 MB) next to the streamed B tiles, so keep them within about 48 MB
+  {
+    const long long rows_bytes = static_cast<long long>(kBlockM) * K;
+    long long gm = (48ll << 20) / rows_bytes;
+    if (gm < 1) gm = 1;
+    const long long mb_all = static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1);
+    if (gm > mb_all) gm = mb_all;
+    p.group_m = static_cast<int>(gm);
+  }
 
   CUtensorMap mA, mB, mC;
   const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;

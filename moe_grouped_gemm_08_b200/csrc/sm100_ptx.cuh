@@ -96,12 +96,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// 3-D tiled load global -> shared with the default L2 policy.
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+// 3-D tiled load global -> shared with an L2 cache policy (from createpolicy).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z,
+                                            uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z)
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "l"(policy)
       : "memory");
 }
 
@@ -205,16 +206,6 @@ __device__ __forceinline__ void pdl_wait_prior_grid() { asm volatile("griddepcon
 // ... and allow the next kernel of the stream to begin its prologue.
 __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// Packed FP32 fused multiply-add (sm_100a): a0 = fma(v0, s, a0) and a1 = fma(v1, s, a1), each
-// lane rounded exactly like fmaf, in one instruction.
-__device__ __forceinline__ void ffma2(float& a0, float& a1, float v0, float v1, float s) {
-  asm("{\n\t.reg .b64 a, v, s;\n\t"
-      "mov.b64 a, {%0, %1};\n\tmov.b64 v, {%2, %3};\n\tmov.b64 s, {%4, %4};\n\t"
-      "fma.rn.f32x2 a, v, s, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
-      : "+f"(a0), "+f"(a1)
-      : "f"(v0), "f"(v1), "f"(s));
 }
 
 // Release + acquire fence at GPU scope (orders this thread's, and by barrier cumulativity the
