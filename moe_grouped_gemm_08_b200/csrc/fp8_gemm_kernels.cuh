@@ -585,6 +585,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int SCALE_CAP = kSwapScaleBytes / (4 * MP);  // units whose scales fit in shared memory
   constexpr int F4 = MP * kBlockM / 4 / NPROMO;          // float4 of a partial tile per thread
   constexpr int PPR = (16 / F4) < 1 ? 1 : 16 / F4;       // partials read per round in the fix-up
+  constexpr int RING_SLOTS = (STAGES * STAGE_BYTES) / (MP * kBlockM * 4);  // partials the idle ring holds
+  static_assert(RING_SLOTS >= 2, "ring slots");
   constexpr uint32_t IDESC = idesc_e4m3_f32(kBlockM, MP);
 
   extern __shared__ uint8_t smem_raw[];
@@ -810,12 +812,51 @@ __global__ void __launch_bounds__(kThreads, 1)
           float4 r[F4];
 #pragma unroll
           for (int i = 0; i < F4; ++i) r[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+          // workspace slot of piece c: the tile's first CTA may hold it as the last segment of its
+          // range (slot 2c+1); every later CTA holds it as its first segment (slot 2c)
+          const int first_slot = sk_slot(c_first, P, U, tu0);
+          auto piece_slot = [&](int c) { return c == c_first ? first_slot : 2 * c; };
+          if (tu0 + kb1 >= u_end) {
+            // The CTA's last segment: its ring is idle (every load consumed, every MMA done), so
+            // the partials are pulled into it with cp.async, RING_SLOTS partials in flight, each
+            // thread copying and reading back only its own float4 positions.  Summation order
+            // is still c_first .. c_last.
+            float4* ring4 = reinterpret_cast<float4*>(smem);
+            const int npieces = c_last - c_first + 1;
+#pragma unroll 1
+            for (int k = 0; k < RING_SLOTS; ++k) {
+              if (k < npieces) {
+                const float4* src = ws4 + static_cast<size_t>(piece_slot(c_first + k)) * (MP * kBlockM / 4) + tid;
+                float4* dst = ring4 + k * F4 * NPROMO + tid;
+#pragma unroll
+                for (int i = 0; i < F4; ++i) cp_async_16(dst + i * NPROMO, src + i * NPROMO);
+              }
+              cp_async_commit();
+            }
+#pragma unroll 1
+            for (int k = 0; k < npieces; ++k) {
+              cp_async_wait<RING_SLOTS - 1>();  // piece k has landed
+              float4* slot = ring4 + (k % RING_SLOTS) * F4 * NPROMO + tid;
+#pragma unroll
+              for (int i = 0; i < F4; ++i) {
+                const float4 a = slot[i * NPROMO];
+                r[i].x += a.x; r[i].y += a.y; r[i].z += a.z; r[i].w += a.w;
+              }
+              if (k + RING_SLOTS < npieces) {
+                const float4* src =
+                    ws4 + static_cast<size_t>(piece_slot(c_first + k + RING_SLOTS)) * (MP * kBlockM / 4) + tid;
+#pragma unroll
+                for (int i = 0; i < F4; ++i) cp_async_16(slot + i * NPROMO, src + i * NPROMO);
+              }
+              cp_async_commit();
+            }
+          } else
           for (int c0 = c_first; c0 <= c_last; c0 += PPR) {
             float4 a[PPR][F4];
 #pragma unroll
             for (int k = 0; k < PPR; ++k) {
               if (c0 + k <= c_last) {
-                const float4* src = ws4 + static_cast<size_t>(sk_slot(c0 + k, P, U, tu0)) * (MP * kBlockM / 4) + tid;
+                const float4* src = ws4 + static_cast<size_t>(piece_slot(c0 + k)) * (MP * kBlockM / 4) + tid;
 #pragma unroll
                 for (int i = 0; i < F4; ++i) a[k][i] = __ldcg(src + i * NPROMO);
               }
