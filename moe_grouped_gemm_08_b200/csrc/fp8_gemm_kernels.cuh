@@ -7,7 +7,8 @@
 // two-level accumulation of the news article's optimisation paragraph and of
 // the turtlesai.it summary).
 //
-// Both kernels use the same warp roles (320 threads):
+// Warp roles (kernel 2: 320 threads; kernel 1: 384 threads, the last four warps being
+// warpgroup 2 of which warps 10-11 idle):
 //   warps 0-7 : promotion + epilogue.  Warp w reads TMEM lanes 32*(w%4)..+31
 //               (the lane quadrant its SM sub-partition can reach) and column
 //               half w/4 of every partial tile.
@@ -21,8 +22,9 @@
 // block kb is being promoted; the FP32 accumulators live in registers.
 //
 // Kernel 1, fp8_gemm_tiled_kernel: persistent CTAs walk 128 x BN output tiles
-//   (dense, M-grouped contiguous, M-grouped masked), m-block fastest.  The
-//   masked walk enumerates only live tiles from masked_m read on the device.
+//   (dense, M-grouped contiguous, M-grouped masked) in groups of m-blocks,
+//   m-block fastest.  The masked walk enumerates only live tiles from masked_m
+//   read on the device.  The epilogue stores bf16 through shared memory with TMA.
 // Kernel 2, fp8_gemm_swap_streamk_kernel (dense, M <= 128, the decode shapes):
 //   swap-AB -- 128 weight rows of B form the MMA's M side and the MP tokens
 //   its N side -- and stream-K: the (n-block, K-block) units are split evenly
