@@ -145,6 +145,15 @@ const char* fg_status_string(fg_status status);
  * an unknown value is ignored. */
 int fg_set_dense_path(int path);
 
+/* Failure injection for tests (process-wide, default 0).  With 1, every kernel of
+ * fp8_gemm_nt that takes the small-M (swap-AB stream-K) path first waits on a barrier
+ * that no one arrives at; the bounded wait runs out after about two seconds, the
+ * kernel aborts cleanly (its other warps leave their waits, copies in flight are
+ * drained, TMEM is freed), writes no output and leaves FG_ERR_TIMEOUT in the device
+ * status word for fg_get_device_status().  Nothing faults or traps, and the context
+ * stays usable.  Returns the previous value.  Not for production use. */
+int fg_debug_set_stall(int enable);
+
 /* Number of GEMM kernel launches the library has issued in this process. */
 uint64_t fg_launch_count(void);
 

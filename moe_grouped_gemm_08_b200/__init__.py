@@ -52,6 +52,8 @@ _lib.fg_status_string.argtypes = [_int]
 _lib.fg_status_string.restype = ctypes.c_char_p
 _lib.fg_set_dense_path.argtypes = [_int]
 _lib.fg_set_dense_path.restype = _int
+_lib.fg_debug_set_stall.argtypes = [_int]
+_lib.fg_debug_set_stall.restype = _int
 _lib.fg_launch_count.argtypes = []
 _lib.fg_launch_count.restype = ctypes.c_uint64
 

@@ -88,6 +88,7 @@ struct SwapParams {
   int M, N, K, ld;
   int num_kb;
   int n_tiles;     // ceil(N / 128)
+  int debug_stall; // test hook: 1 = the MMA thread first waits on a barrier no one arrives at
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -664,6 +665,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
+      // Failure-injection hook for tests: mma_done completes its first phase only with the commit
+      // below, so this bounded wait runs out, raises the abort flag and exercises the abort path.
+      if (p.debug_stall) mbar_wait(mma_done, 0, abort_flag, kWaitLimitNs);
       for (int u = u_begin; u < u_end; ++u) {
         if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
         if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) break;

@@ -38,6 +38,7 @@ std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 std::atomic<int> g_dense_path{0};
+std::atomic<int> g_debug_stall{0};
 std::atomic<uint64_t> g_launches{0};
 
 // tiled kernel configuration: 128 x 192 output tiles, 4-stage ring (overridable when building)
@@ -46,6 +47,9 @@ std::atomic<uint64_t> g_launches{0};
 #endif
 #ifndef FG_TILED_STAGES
 #define FG_TILED_STAGES 4
+#endif
+#ifndef FG_TILED_GROUP_MB
+#define FG_TILED_GROUP_MB 48  // L2 budget (MB) for the A rows of one group of m-blocks
 #endif
 constexpr int kTiledBN = FG_TILED_BN;
 constexpr int kTiledStages = FG_TILED_STAGES;
@@ -202,10 +206,10 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
   p.m_blocks = (M + kBlockM - 1) / kBlockM;
   p.n_blocks = (N + BN - 1) / BN;
   // m-blocks per group of the tile walk: a group's A rows (128 * K bytes per m-block) should stay
-  // in L2 (126 MB) next to the streamed B tiles, so keep them within about 48 MB
+  // in L2 (126 MB) next to the streamed B tiles, so keep them within FG_TILED_GROUP_MB
   {
     const long long rows_bytes = static_cast<long long>(kBlockM) * K;
-    long long gm = (48ll << 20) / rows_bytes;
+    long long gm = (static_cast<long long>(FG_TILED_GROUP_MB) << 20) / rows_bytes;
     if (gm < 1) gm = 1;
     const long long mb_all = static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1);
     if (gm > mb_all) gm = mb_all;
@@ -243,6 +247,7 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
   p.ld = fg_sfa_ld(M);
   p.num_kb = (K + kBlockK - 1) / kBlockK;
   p.n_tiles = (N + kBlockM - 1) / kBlockM;
+  p.debug_stall = g_debug_stall.load(std::memory_order_relaxed);
   if (p.n_tiles > kCounterCapacity) return FG_ERR_UNSUPPORTED;
 
   CUtensorMap mW, mT;
@@ -315,6 +320,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.ld = fg_sfa_ld(M);
   p.num_kb = (K + kBlockK - 1) / kBlockK;
   p.n_tiles = (N + kBlockM - 1) / kBlockM;
+  p.debug_stall = 0;
   if (p.n_tiles > kNoAllocCounters) return FG_ERR_UNSUPPORTED;
   // the counters must start at zero; the kernel leaves them at zero, but a call that gave up a
   // wait may not have, so clear the ones this call uses (a memset, no allocation)
@@ -395,6 +401,8 @@ int fg_set_dense_path(int path) {
 }
 
 uint64_t fg_launch_count(void) { return g_launches.load(); }
+
+int fg_debug_set_stall(int enable) { return g_debug_stall.exchange(enable ? 1 : 0); }
 
 fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
                       int K, void* stream) {
