@@ -90,7 +90,8 @@ def record_traffic(csv_path: str, workload: str) -> None:
         if len(r) != len(h) or not r[col["Metric Name"]].startswith("dram__bytes_"):
             continue
         name = r[col["Kernel Name"]]
-        kern = next((k for k in ("fp8_gemm_swap_streamk_kernel", "fp8_gemm_tiled_kernel") if k in name), None)
+        kern = next((k for k in ("fp8_gemm_swap_streamk_kernel", "fp8_gemm_tiled_kernel", "fp8_gemm_pair_kernel")
+                     if k in name), None)
         if kern is None:
             continue
         v = float(r[col["Metric Value"]].replace(",", "")) * scale.get(r[col["Metric Unit"]], 1)
@@ -156,10 +157,18 @@ def work_of(case):
     return flops, byt, M * K + N * K + 2 * M * N
 
 
+KERNEL_PATH = 0  # the kernel selection bench.py runs with (--path)
+
+
 def kernel_name(case) -> str:
-    if case["kind"] == "dense" and case["M"] <= 128:
-        return "fp8_gemm_swap_streamk_kernel"
-    return "fp8_gemm_tiled_kernel"
+    """The library kernel a case runs on under the selection KERNEL_PATH (fg_set_dense_path)."""
+    if case["kind"] == "contiguous":
+        return "fp8_gemm_tiled_kernel"
+    if KERNEL_PATH == 3:
+        return "fp8_gemm_pair_kernel"
+    if case["kind"] == "masked" or KERNEL_PATH == 1:
+        return "fp8_gemm_tiled_kernel"
+    return "fp8_gemm_swap_streamk_kernel" if (KERNEL_PATH == 2 or case["M"] <= 128) else "fp8_gemm_tiled_kernel"
 
 
 def upload(case, dev):
@@ -363,6 +372,9 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     fg.init(local)
+    global KERNEL_PATH
+    KERNEL_PATH = args.path
+    fg.set_dense_path(args.path)
     name, wl = workload_list(args.workload, args.shape)
     cases = [make_case(w) for w in wl]
     works = [work_of(c) for c in cases]
@@ -526,7 +538,8 @@ def run_ours(args, rank, world, local):
             "data": "synthetic",
             "config": {"workload": name, "shapes": [w["name"] for w in wl],
                        "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
-                       "graph": "each step replayed from a CUDA graph", "parallelism": f"replicas x{world}"},
+                       "graph": "each step replayed from a CUDA graph", "parallelism": f"replicas x{world}",
+                       "kernel_path": args.path},
             "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
             "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
             "roofline": roof,
@@ -554,6 +567,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="kernel selection (fg_set_dense_path): 0 automatic, 1 one-CTA tiled, "
+                         "2 swap-AB stream-K, 3 CTA pair")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

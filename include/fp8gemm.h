@@ -139,10 +139,13 @@ fg_status fg_get_device_status(void* stream);
 /* Human-readable name of a status code (static storage). */
 const char* fg_status_string(fg_status status);
 
-/* Dense-path selection, process-wide: 0 = automatic (M <= 128 takes the
- * swap-AB stream-K kernel, larger M the tiled kernel), 1 = always tiled,
- * 2 = always swap-AB stream-K (requires M <= 128).  Returns the previous value;
- * an unknown value is ignored. */
+/* Kernel selection, process-wide: 0 = automatic (dense M <= 128 takes the
+ * swap-AB stream-K kernel, everything else the one-CTA tiled kernel), 1 = the
+ * one-CTA tiled kernel for every dense call, 2 = always swap-AB stream-K for
+ * dense calls (requires M <= 128), 3 = the CTA-pair kernel (tcgen05 cta_group::2,
+ * 256-row tiles over two SMs) for dense and masked calls.  The contiguous layout
+ * always takes the one-CTA tiled kernel.  Returns the previous value; an unknown
+ * value is ignored. */
 int fg_set_dense_path(int path);
 
 /* Failure injection for tests (process-wide, default 0).  With 1, every kernel of

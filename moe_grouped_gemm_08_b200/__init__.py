@@ -92,7 +92,8 @@ def sfa_ld(m: int) -> int:
 
 
 def set_dense_path(path: int) -> int:
-    """0 automatic, 1 tiled kernel, 2 swap-AB stream-K kernel (M <= 128). Returns the old value."""
+    """0 automatic, 1 one-CTA tiled kernel (dense), 2 swap-AB stream-K (dense, M <= 128),
+    3 CTA-pair kernel (dense and masked). Returns the old value."""
     return int(_lib.fg_set_dense_path(int(path)))
 
 

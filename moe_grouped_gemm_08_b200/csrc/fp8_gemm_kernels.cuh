@@ -146,7 +146,8 @@ __device__ __forceinline__ void tile_coords(int t, int mblocks, int n_blocks, in
   mb = gm0 + (rem - nb * gm);
 }
 
-template <int MODE>
+// ROWS: rows of an m-block (128, or 256 for the CTA-pair kernel); s_prefix counts such blocks.
+template <int MODE, int ROWS = kBlockM>
 __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* s_prefix, int live_mblocks, int t,
                                                int BN) {
   TileInfo ti;
@@ -160,12 +161,12 @@ __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* 
     }
     ti.live = 1;
     ti.g = lo;
-    ti.m0 = (lm - s_prefix[lo]) * kBlockM;
+    ti.m0 = (lm - s_prefix[lo]) * ROWS;
     ti.n0 = nb * BN;
   } else {
     int mb, nb;
     tile_coords(t, p.m_blocks, p.n_blocks, p.group_m, mb, nb);
-    ti.m0 = mb * kBlockM;
+    ti.m0 = mb * ROWS;
     ti.n0 = nb * BN;
     if (MODE == kContiguous) {
       const int g = __ldg(p.m_indices + ti.m0);
@@ -551,6 +552,347 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status);
+}
+
+// ============================================================================
+// Kernel 3: CTA-pair tiled (dense M > 128, masked)
+// ============================================================================
+// The two CTAs of a cluster compute one 256 x BN output tile with tcgen05.mma.cta_group::2: CTA
+// r loads A rows m0 + 128 r .. +127 and B rows n0 + r BN/2 .. +BN/2-1 of every K block into its
+// own ring, the leader (rank 0) issues the pair MMAs (M = 256, N = BN), and the TMEM of CTA r
+// holds rows m0 + 128 r .. +127 x BN columns, promoted and stored by CTA r as in kernel 1.  Each
+// SM thus reads half of the B tile per K block instead of all of it.
+// Barriers: full[s] of the leader counts the bytes of both CTAs (armed by the leader's producer);
+// empty[s], tfull[b] and mma_done of both CTAs are arrived by the leader's multicast commits;
+// tempty[b] of the leader counts the promotion warps of both CTAs.  Cluster barriers only right
+// after set-up and right before teardown, which every thread of both CTAs reaches; every other
+// wait is bounded.
+template <int BN, int STAGES, int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
+    fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
+  static_assert(MODE != kContiguous, "a pair tile needs both 128-row halves in one group");
+  constexpr int COLS = BN / 2;    // columns per promotion thread
+  constexpr int NCH = COLS / 32;  // 32-column TMEM loads (and store boxes) per thread
+  static_assert(COLS % 32 == 0 && BN <= 256, "BN");
+  constexpr int PAIR_ROWS = 2 * kBlockM;
+  constexpr int A_BYTES = kBlockM * kBlockK;   // this CTA's 128 rows of A
+  constexpr int B_BYTES = COLS * kBlockK;      // this CTA's half of the B tile
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int NUM_TBUF = 512 / BN;
+  constexpr uint32_t TMEM_COLS = 512;
+  constexpr int CHUNK_FLOATS = kSaChunk * kBlockM + 2 * kSaChunk;
+  constexpr uint32_t IDESC = idesc_e4m3_f32(PAIR_ROWS, BN);
+  constexpr int WARP_STORE_BYTES = NCH * kStoreBoxBytes;
+  constexpr uint16_t kBoth = 0x3;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_1024(smem_raw);  // same offsets in both CTAs: the pair MMA relies on it
+  uint8_t* s_out = smem + STAGES * STAGE_BYTES;
+  float* s_scale = reinterpret_cast<float*>(s_out + kPromoWarps * WARP_STORE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + 2 * CHUNK_FLOATS);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + NUM_TBUF;
+  uint64_t* mma_done = tempty + NUM_TBUF;
+  uint64_t* pbar = mma_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int num_pairs = static_cast<int>(gridDim.x >> 1);
+
+  if (warp == kProducerWarp && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    prefetch_tmap(&tmC);
+    for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 2 * kPromoWarps); }
+    mbar_init(mma_done, 1);
+    mbar_init(pbar, kPromoWarps * 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) { tmem_alloc_pair(tmem_slot, TMEM_COLS); tmem_relinquish_pair(); }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers are initialised before either CTA signals the other
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_prior_grid();
+  pdl_launch_dependents();
+
+  if (MODE == kMasked) {
+    if (warp == 0) {
+      // live 256-row blocks per group, exclusive prefix in s_prefix[0..G]
+      int carry = 0;
+      if (lane == 0) s_prefix[0] = 0;
+      for (int base = 0; base < p.G; base += 32) {
+        const int g = base + lane;
+        int v = 0;
+        if (g < p.G) {
+          int cnt = __ldg(p.masked_m + g);
+          cnt = cnt < 0 ? 0 : (cnt > p.M ? p.M : cnt);
+          v = (cnt + PAIR_ROWS - 1) / PAIR_ROWS;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        if (g < p.G) s_prefix[g + 1] = carry + v;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+      }
+    }
+    __syncthreads();
+  }
+
+  int num_tiles, live_blocks = 1;
+  if (MODE == kMasked) {
+    live_blocks = s_prefix[p.G];
+    num_tiles = live_blocks * p.n_blocks;
+  } else {
+    num_tiles = p.m_blocks * p.n_blocks;  // m_blocks counts 256-row blocks here
+  }
+
+  if (warp >= kPromoWarps) {
+    // ================================================ warpgroup 2: producer, MMA, idle warps
+    reg_dealloc<kCtrlRegs>();
+    if (warp == kProducerWarp && lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      const uint32_t full_leader = mapa_shared(smem_addr(full), 0);
+      const uint64_t pol_a = l2_policy_evict_last();
+      const uint64_t pol_b = l2_policy_evict_first();
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+        const TileInfo ti = tiled_tile<MODE, PAIR_ROWS>(p, s_prefix, live_blocks, t, BN);
+        const int ga = (MODE == kMasked) ? ti.g : 0;
+        const int gb = (MODE == kDense) ? 0 : ti.g;
+        const int a_row = ti.m0 + static_cast<int>(rank) * kBlockM;
+        const int b_row = ti.n0 + static_cast<int>(rank) * COLS;
+        for (int kb = 0; kb < p.num_kb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          uint8_t* st = smem + stage * STAGE_BYTES;
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          tma_load_3d_pair(st, &tmA, full_leader + stage * 8, kb * kBlockK, a_row, ga, pol_a);
+          tma_load_3d_pair(st + A_BYTES, &tmB, full_leader + stage * 8, kb * kBlockK, b_row, gb, pol_b);
+          ++issued;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // copies still in flight: the leader sees them complete on its own barriers; the peer's
+        // land on the leader's barriers, so it gives them a fixed grace period instead
+        if (leader) {
+          const uint32_t first = issued > STAGES ? issued - STAGES : 0;
+          for (uint32_t i = first; i < issued; ++i) mbar_drain(&full[i % STAGES], (i / STAGES) & 1u);
+        } else {
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 50000ull) {
+          }
+        }
+      }
+    } else if (warp == kMmaWarp && lane == 0) {
+      if (leader) {
+        uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
+        bool ok = true;
+        for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+          for (int kb = 0; kb < p.num_kb; ++kb) {
+            if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+            if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t d = tmem_base + tb * BN;
+            const uint32_t st = smem_addr(smem + stage * STAGE_BYTES);
+            const uint64_t adesc = smem_desc_k128_sw128(st);
+            const uint64_t bdesc = smem_desc_k128_sw128(st + A_BYTES);
+#pragma unroll
+            for (int j = 0; j < kBlockK / 32; ++j)
+              mma_f8_pair(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+            mma_commit_pair(&empty[stage], kBoth);
+            mma_commit_pair(&tfull[tb], kBoth);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+          }
+        }
+        mma_commit_pair(mma_done, kBoth);  // arrives on both CTAs once every pair MMA has finished
+      }
+    }
+  } else {
+    // ================================================ warpgroups 0-1: promotion + epilogue
+    reg_alloc<kPromoRegs>();
+    const int q = warp & 3;
+    const int h = warp >> 2;
+    const int row = q * 32 + lane;
+    const int tid = threadIdx.x;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const int n_chunks = (p.num_kb + kSaChunk - 1) / kSaChunk;
+    const uint32_t tempty_leader = mapa_shared(smem_addr(tempty), 0);
+    uint8_t* s_w = s_out + warp * WARP_STORE_BYTES;
+    bool stores_pending = false;
+    uint32_t tb = 0, tphase = 0, pphase = 0;
+    bool ok = true;
+
+    // this CTA's half of the pair tile t
+    auto my_tile = [&](int tt) {
+      TileInfo ti = tiled_tile<MODE, PAIR_ROWS>(p, s_prefix, live_blocks, tt, BN);
+      ti.m0 += static_cast<int>(rank) * kBlockM;
+      return ti;
+    };
+    int t = pair;
+    TileInfo ti;
+    ti.live = 0;
+    if (t < num_tiles) ti = my_tile(t);
+    ScaleChunkRegs nxt;
+    int buf = 0;
+    if (t < num_tiles) {
+      load_scale_chunk<MODE>(p, ti, 0, tid, nxt);
+      store_scale_chunk(s_scale, tid, nxt);
+      ok = group_sync(pbar, pphase, abort_flag);
+    }
+    while (t < num_tiles && ok) {
+      const int t_next = t + num_pairs;
+      TileInfo ti_next;
+      ti_next.live = 0;
+      if (t_next < num_tiles) ti_next = my_tile(t_next);
+      const int m = ti.m0 + row;
+      uint32_t hi_mask = 0;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+        hi_mask |= static_cast<uint32_t>((ti.n0 + h * COLS + 32 * i) / kBlockK - ti.n0 / kBlockK) << i;
+
+      float2 acc[COLS / 2];
+#pragma unroll
+      for (int j = 0; j < COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+
+      for (int c = 0; c < n_chunks && ok; ++c) {
+        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, nxt);
+        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, nxt);
+        const float* sa = s_scale + buf * CHUNK_FLOATS + row;
+        const float* sb = s_scale + buf * CHUNK_FLOATS + kSaChunk * kBlockM;
+        const int kb_end = (c + 1) * kSaChunk < p.num_kb ? (c + 1) * kSaChunk : p.num_kb;
+        for (int kb = c * kSaChunk; kb < kb_end; ++kb) {
+          const int kl = kb - c * kSaChunk;
+          const float sav = sa[kl * kBlockM];
+          const float s0 = sav * sb[kl];
+          const float s1 = sav * sb[kSaChunk + kl];
+          if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
+          uint32_t v[NCH][32];
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) tmem_ld_32x32b_x32(taddr + 32 * i, v[i]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader + tb * 8);
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const float s = ((hi_mask >> i) & 1u) ? s1 : s0;
+            const float2 s2 = make_float2(s, s);
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              acc[16 * i + j] = __ffma2_rn(make_float2(__uint_as_float(v[i][2 * j]), __uint_as_float(v[i][2 * j + 1])),
+                                           s2, acc[16 * i + j]);
+          }
+          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+        }
+        if (!ok) break;
+        const int nbuf = buf ^ 1;
+        if (c + 1 < n_chunks || t_next < num_tiles) store_scale_chunk(s_scale + nbuf * CHUNK_FLOATS, tid, nxt);
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        buf = nbuf;
+      }
+      if (!ok) break;
+
+      // epilogue, as in kernel 1
+      bool store_row = m < p.M;
+      if (MODE == kMasked) {
+        int cnt = __ldg(p.masked_m + ti.g);
+        cnt = cnt > p.M ? p.M : cnt;
+        store_row = m < cnt;
+      }
+      const int nbase = ti.n0 + h * COLS;
+      if (__all_sync(0xffffffffu, store_row)) {
+        if (stores_pending) {
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
+        }
+        const uint32_t sw = static_cast<uint32_t>((lane >> 1) & 3);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+          uint8_t* box_row = s_w + i * kStoreBoxBytes + lane * 64;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float2* a = acc + 16 * i + 4 * c;
+            uint4 val;
+            val.x = pack_bf16x2(a[0].x, a[0].y);
+            val.y = pack_bf16x2(a[1].x, a[1].y);
+            val.z = pack_bf16x2(a[2].x, a[2].y);
+            val.w = pack_bf16x2(a[3].x, a[3].y);
+            *reinterpret_cast<uint4*>(box_row + ((c ^ sw) << 4)) = val;
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int y = ti.m0 + q * 32;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            if (nbase + 32 * i < p.N) {
+              if (MODE == kMasked) tma_store_3d(&tmC, s_w + i * kStoreBoxBytes, nbase + 32 * i, y, ti.g);
+              else tma_store_2d(&tmC, s_w + i * kStoreBoxBytes, nbase + 32 * i, y);
+            }
+          }
+          bulk_commit_group();
+        }
+        stores_pending = true;
+      } else if (store_row) {
+        __nv_bfloat16* crow = (MODE == kMasked) ? p.C + (static_cast<size_t>(ti.g) * p.M + m) * p.N
+                                                : p.C + static_cast<size_t>(m) * p.N;
+#pragma unroll
+        for (int j = 0; j < COLS; j += 8) {
+          if (nbase + j < p.N) {
+            const float2* a = acc + j / 2;
+            uint4 val;
+            val.x = pack_bf16x2(a[0].x, a[0].y);
+            val.y = pack_bf16x2(a[1].x, a[1].y);
+            val.z = pack_bf16x2(a[2].x, a[2].y);
+            val.w = pack_bf16x2(a[3].x, a[3].y);
+            *reinterpret_cast<uint4*>(crow + nbase + j) = val;
+          }
+        }
+      }
+      t = t_next;
+      ti = ti_next;
+    }
+    if (stores_pending && lane == 0) bulk_wait_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    // both CTAs: every pair MMA (which read this CTA's ring and wrote its TMEM) has finished; the
+    // promotion above consumed every result, so this wait is short unless the CTA aborted
+    if (lane == 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait_cluster(mma_done, 0)) {
+        if (global_timer_ns() - t0 > kWaitLimitNs) { *abort_flag = 1; break; }
+      }
+    }
+    __syncwarp();
+  }
+  cluster_sync_all();  // neither CTA touches the other's barriers, ring or TMEM any more
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
   if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status);
 }

@@ -53,6 +53,9 @@ std::atomic<uint64_t> g_launches{0};
 #endif
 constexpr int kTiledBN = FG_TILED_BN;
 constexpr int kTiledStages = FG_TILED_STAGES;
+// CTA-pair kernel: 256 x 192 tiles per pair, each CTA's stage = 128 A rows + 96 B rows
+constexpr int kPairBN = 192;
+constexpr int kPairStages = 5;
 
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
@@ -62,6 +65,14 @@ constexpr size_t tiled_smem_bytes() {
          4 * (fg::kMaskedMaxGroups + 1) /*masked prefix*/;
 }
 static_assert(tiled_smem_bytes<kTiledBN, kTiledStages>() <= 227 * 1024, "tiled kernel shared memory");
+
+template <int BN, int STAGES>
+constexpr size_t pair_smem_bytes() {
+  return 1024 + static_cast<size_t>(STAGES) * (kBlockM + BN / 2) * kBlockK +
+         static_cast<size_t>(fg::kPromoWarps) * (BN / 64) * fg::kStoreBoxBytes +
+         2 * (fg::kSaChunk * kBlockM + 2 * fg::kSaChunk) * 4 + 256 + 4 * (fg::kMaskedMaxGroups + 1);
+}
+static_assert(pair_smem_bytes<kPairBN, kPairStages>() <= 227 * 1024, "pair kernel shared memory");
 
 template <int MP>
 constexpr int swap_stages() {
@@ -230,6 +241,82 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
                                                               fg::kTiledThreads, fg::kTiledLaunchRegs);
 }
 
+// Largest number of CTA pairs of the pair kernel that can be resident at once (queried once per
+// device and kernel; clusters must fit inside a GPC, so this can be below #SMs / 2).
+template <auto KERNEL>
+int pair_capacity(int sms, size_t smem) {
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return sms / 2;
+  int v = cached[dev].load(std::memory_order_acquire);
+  if (v > 0) return v;
+  // the query needs the kernel's opt-in shared-memory size in place
+  if (cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return sms / 2;
+  }
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
+  cfg.blockDim = dim3(fg::kTiledThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, KERNEL, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sms / 2;
+  }
+  cached[dev].store(n, std::memory_order_release);
+  return n;
+}
+
+template <int MODE>
+fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                   const int* masked_m, int M, int G, int N, int K, cudaStream_t stream) {
+  constexpr int BN = kPairBN;
+  constexpr int STAGES = kPairStages;
+  constexpr auto KERNEL = fg::fp8_gemm_pair_kernel<BN, STAGES, MODE>;
+  constexpr size_t SMEM = pair_smem_bytes<BN, STAGES>();
+  fg::TiledParams p;
+  p.sfa = sfa;
+  p.sfb = sfb;
+  p.C = static_cast<__nv_bfloat16*>(C);
+  p.m_indices = nullptr;
+  p.masked_m = masked_m;
+  p.status = st->status;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.G = G;
+  p.ld = fg_sfa_ld(M);
+  p.num_kb = (K + kBlockK - 1) / kBlockK;
+  p.num_nb = (N + kBlockK - 1) / kBlockK;
+  p.m_blocks = (M + 2 * kBlockM - 1) / (2 * kBlockM);  // 256-row blocks
+  p.n_blocks = (N + BN - 1) / BN;
+  {
+    const long long rows_bytes = 2ll * kBlockM * K;
+    long long gm = (static_cast<long long>(FG_TILED_GROUP_MB) << 20) / rows_bytes;
+    if (gm < 1) gm = 1;
+    const long long mb_all = static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1);
+    if (gm > mb_all) gm = mb_all;
+    p.group_m = static_cast<int>(gm);
+  }
+
+  CUtensorMap mA, mB, mC;
+  const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;
+  const uint64_t groupsB = (MODE == fg::kDense) ? 1 : static_cast<uint64_t>(G);
+  if (!encode_fp8_map(&mA, A, K, M, groupsA, kBlockM)) return FG_ERR_CUDA;
+  if (!encode_fp8_map(&mB, B, K, N, groupsB, BN / 2)) return FG_ERR_CUDA;
+  if (!encode_bf16_store_map(&mC, C, N, M, groupsA, MODE == fg::kMasked)) return FG_ERR_CUDA;
+
+  const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
+  const int cap = pair_capacity<KERNEL>(st->sms, SMEM);
+  const int pairs = static_cast<int>(tiles < cap ? tiles : cap);
+  void* args[4] = {&mA, &mB, &mC, &p};
+  return launch<KERNEL>(dim3(static_cast<unsigned>(2 * pairs)), SMEM, stream, args, fg::kTiledThreads,
+                        fg::kTiledLaunchRegs);
+}
+
 template <int MP>
 fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    int M, int N, int K, cudaStream_t stream) {
@@ -396,7 +483,7 @@ int fg_m_alignment(void) { return kBlockM; }
 int fg_sfa_ld(int M) { return M <= 0 ? 0 : (M + 3) / 4 * 4; }
 
 int fg_set_dense_path(int path) {
-  if (path < 0 || path > 2) return g_dense_path.load();
+  if (path < 0 || path > 3) return g_dense_path.load();
   return g_dense_path.exchange(path);
 }
 
@@ -423,6 +510,7 @@ fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const floa
     if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs);
     return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs);
   }
+  if (path == 3) return run_pair<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, M, 1, N, K, cs);
   return run_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs);
 }
 
@@ -456,6 +544,8 @@ fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B
     return FG_ERR_UNSUPPORTED;
   DeviceState* st = state_for_current(&s);
   if (!st) return s;
+  if (g_dense_path.load() == 3)
+    return run_pair<fg::kMasked>(st, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K, static_cast<cudaStream_t>(stream));
   return run_tiled<fg::kMasked>(st, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
                                 static_cast<cudaStream_t>(stream));
 }

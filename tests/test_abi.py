@@ -44,7 +44,8 @@ def test_queries():
 def test_dense_path_switch():
     old = fg.set_dense_path(1)
     assert fg.set_dense_path(2) == 1
-    assert fg.set_dense_path(7) == 2  # ignored
+    assert fg.set_dense_path(3) == 2
+    assert fg.set_dense_path(7) == 3  # ignored
     fg.set_dense_path(old)
 
 

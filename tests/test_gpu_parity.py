@@ -69,7 +69,7 @@ ODD = [(1, 8, 16), (7, 136, 272), (33, 4104, 2048), (64, 264, 640), (100, 2112, 
 def test_dense_odd_shapes(fg, M, N, K):
     case = synth.dense_case(100 + M, M, N, K, row_scaled=True)
     ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
-    for path in ([1, 2] if M <= 128 else [1]):
+    for path in ([1, 2, 3] if M <= 128 else [1, 3]):  # 1 tiled, 2 swap-AB stream-K, 3 CTA pair
         close(run_dense(fg, case, path), ref, f"odd {M}x{N}x{K} path={path}")
 
 
@@ -87,8 +87,9 @@ def test_prefill_sampled_rows(fg, w):
     case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"])
     rows = sample_rows(w["M"], 40, w["seed"])
     ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"], rows=rows)
-    got = run_dense(fg, case, 0)
-    close(got[rows], ref, w["name"])
+    for path in (0, 3):  # the one-CTA tiled kernel (automatic) and the CTA-pair kernel
+        got = run_dense(fg, case, path)
+        close(got[rows], ref, f"{w['name']} path={path}")
 
 
 @pytest.mark.parametrize("idx", [0, 6, 8])
@@ -169,8 +170,17 @@ def check_masked(got, case, what):
         assert np.all(got[g, v:] == 0xFFFF), f"{what}: rows past masked_m[{g}]={v} were written"
 
 
+@pytest.mark.parametrize("path", [0, 3], ids=["tiled", "pair"])
 @pytest.mark.parametrize("w", workloads.masked(), ids=lambda w: w["name"])
-def test_masked_under_cuda_graph(fg, w):
+def test_masked_under_cuda_graph(fg, w, path):
+    old_path = fg.set_dense_path(path)  # the masked entry point takes the CTA-pair kernel with 3
+    try:
+        _masked_under_cuda_graph(fg, w)
+    finally:
+        fg.set_dense_path(old_path)
+
+
+def _masked_under_cuda_graph(fg, w):
     case = synth.masked_case(w["seed"], w["G"], w["Mmax"], w["N"], w["K"])
     A, sfa, B, sfb, mm = masked_dev(case)
     C = canary_like((w["G"], w["Mmax"], w["N"]))
@@ -203,7 +213,16 @@ def test_masked_under_cuda_graph(fg, w):
     del graph
 
 
-def test_masked_counts_edge_cases(fg):
+@pytest.mark.parametrize("path", [0, 3], ids=["tiled", "pair"])
+def test_masked_counts_edge_cases(fg, path):
+    old_path = fg.set_dense_path(path)
+    try:
+        _masked_counts_edge_cases(fg)
+    finally:
+        fg.set_dense_path(old_path)
+
+
+def _masked_counts_edge_cases(fg):
     case = synth.masked_case(51, 3, 200, 136, 256, masked_m=[0, 0, 0])
     A, sfa, B, sfb, mm = masked_dev(case)
     C = canary_like((3, 200, 136))
