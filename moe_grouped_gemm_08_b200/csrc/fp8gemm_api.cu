@@ -54,8 +54,14 @@ std::atomic<uint64_t> g_launches{0};
 constexpr int kTiledBN = FG_TILED_BN;
 constexpr int kTiledStages = FG_TILED_STAGES;
 // CTA-pair kernel: 256 x 192 tiles per pair, each CTA's stage = 128 A rows + 96 B rows
-constexpr int kPairBN = 192;
-constexpr int kPairStages = 5;
+#ifndef FG_PAIR_BN
+#define FG_PAIR_BN 192
+#endif
+#ifndef FG_PAIR_STAGES
+#define FG_PAIR_STAGES 5
+#endif
+constexpr int kPairBN = FG_PAIR_BN;
+constexpr int kPairStages = FG_PAIR_STAGES;
 
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
