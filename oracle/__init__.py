@@ -57,6 +57,9 @@ def load(path) -> ctypes.CDLL:
     lib.oracle_grouped_masked.argtypes = [vp, vp, c_long, vp, vp, vp, c_int, c_int,
                                           c_int, c_int, vp, vp]
     lib.oracle_num_threads.restype = c_int
+    lib.oracle_e4m3_encode_array.argtypes = [vp, c_long, vp]
+    lib.oracle_quantize_rows.argtypes = [vp, c_int, c_int, c_int, vp, vp, c_long]
+    lib.oracle_quantize_blocks.argtypes = [vp, c_int, c_int, c_int, vp, vp]
     return lib
 
 
@@ -160,3 +163,42 @@ def grouped_masked(A, sfa, B, sfb, masked_m, C=None, want_acc: bool = False):
     _lib().oracle_grouped_masked(_p(A), _p(sfa), ld, _p(B), _p(sfb), _p(mm), G, Mmax, N, K,
                                  _p(C), _p(acc))
     return (C, acc) if want_acc else C
+
+
+# ---------------------------------------------------------------------------- the cast step
+def e4m3_encode(v) -> np.ndarray:
+    """e4m3 codes (uint8) of finite fp32 values: round to nearest, ties to even, saturating."""
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _lib().oracle_e4m3_encode_array(_p(v), int(v.size), _p(out))
+    return out
+
+
+def quantize_rows(X_bits, ld=None):
+    """A side of the cast: X_bits bf16 bit patterns [M,K] or [G,M,K] -> (codes of the same shape,
+    sfa [KB, ld] or [G, KB, ld]); one fp32 scale per 1x128 block of a row, column-major."""
+    X = _c(X_bits, np.uint16)
+    squeeze = X.ndim == 2
+    if squeeze:
+        X = X[None]
+    G, M, K = X.shape
+    KB = (K + 127) // 128
+    ld = ld if ld is not None else (M + 3) // 4 * 4
+    Q = np.empty(X.shape, dtype=np.uint8)
+    sfa = np.zeros((G, KB, ld), dtype=np.float32)
+    _lib().oracle_quantize_rows(_p(X), G, M, K, _p(Q), _p(sfa), ld)
+    return (Q[0], sfa[0]) if squeeze else (Q, sfa)
+
+
+def quantize_blocks(X_bits):
+    """B side of the cast: X_bits bf16 bit patterns [N,K] or [G,N,K] -> (codes, sfb [NB,KB] or
+    [G,NB,KB]); one fp32 scale per 128x128 block."""
+    X = _c(X_bits, np.uint16)
+    squeeze = X.ndim == 2
+    if squeeze:
+        X = X[None]
+    G, N, K = X.shape
+    Q = np.empty(X.shape, dtype=np.uint8)
+    sfb = np.empty((G, (N + 127) // 128, (K + 127) // 128), dtype=np.float32)
+    _lib().oracle_quantize_blocks(_p(X), G, N, K, _p(Q), _p(sfb))
+    return (Q[0], sfb[0]) if squeeze else (Q, sfb)

@@ -32,6 +32,9 @@
  * only roundings are the fp64 scale multiply, the fp64 accumulation over kb
  * (in ascending kb order) and the single final rounding to bf16.
  *
+ * It also defines the cast step that produces those inputs from BF16 values
+ * (oracle_quantize_rows / oracle_quantize_blocks, see below).
+ *
  * Build: plain C11, -ffp-contract=off, OpenMP over output rows.
  */
 #include <math.h>
@@ -204,6 +207,113 @@ void oracle_grouped_masked(const uint8_t *A, const float *sfa, long ld,
                B + (size_t)g * N * K, sfb + (size_t)g * NB * KB, N, K,
                C + ((size_t)g * Mmax + m) * N,
                acc ? acc + ((size_t)g * Mmax + m) * N : NULL);
+    }
+}
+
+/* ---------------------------------------------------------------------------
+ * The cast step before the GEMM: BF16 values to e4m3 codes with fine-grained
+ * fp32 scales.  The pages leave this step to the user (turtlesai.it summary:
+ * the LHS scales must be laid out for aligned TMA loads, with the FP8 casting
+ * done separately; news article, senqingzn.com: fine-grained scaling).  The
+ * reading taken here, per block (1 x 128 of a row for A, 128 x 128 for B):
+ *   amax  = max |x| over the block (fp32; bf16 -> fp32 is exact)
+ *   scale = amax / 448 in fp32 (one IEEE round-to-nearest division), or 1 if
+ *           amax == 0
+ *   code  = e4m3 round-to-nearest-even of the fp32 quotient x / scale,
+ *           saturating at +-448 (448 is the largest finite e4m3 value)
+ * ------------------------------------------------------------------------- */
+
+/* e4m3 code of the finite fp32 value v: the nearest of the 127 non-negative
+ * finite magnitudes of the decode table (increasing with the code), ties to
+ * the even code (mantissa LSB 0), magnitudes above 448 clamped to 448. */
+uint8_t oracle_e4m3_encode(float v) {
+    const double *dec = dec_table();
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a >= dec[0x7E]) return sign | 0x7E;
+    int lo = 0, hi = 0x7E;                 /* dec[lo] <= a < dec[hi] */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (dec[mid] <= a) lo = mid; else hi = mid;
+    }
+    const double dl = a - dec[lo], dh = dec[hi] - a;
+    int c;
+    if (dl < dh) c = lo;
+    else if (dh < dl) c = hi;
+    else c = (lo % 2 == 0) ? lo : hi;      /* tie: even mantissa */
+    return sign | (uint8_t)c;
+}
+
+void oracle_e4m3_encode_array(const float *v, long n, uint8_t *out) {
+    for (long i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(v[i]);
+}
+
+static float bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static float block_scale(float amax) {
+    volatile float s = amax / 448.0f;      /* one fp32 division */
+    return amax == 0.0f ? 1.0f : s;
+}
+
+/* A side: X is [G][M][K] bf16 (bit patterns), Q the e4m3 codes in the same
+ * layout, sfa the scales [G][ceil(K/128)][ld], ld >= M (rows M..ld-1 of each
+ * column are not written). */
+void oracle_quantize_rows(const uint16_t *X, int G, int M, int K, uint8_t *Q, float *sfa, long ld) {
+    const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
+    long rows = (long)G * M;
+    #pragma omp parallel for schedule(static)
+    for (long r = 0; r < rows; ++r) {
+        const int g = (int)(r / M), m = (int)(r % M);
+        const uint16_t *x = X + (size_t)r * K;
+        uint8_t *q = Q + (size_t)r * K;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int k0 = kb * ORC_BLOCK, k1 = (k0 + ORC_BLOCK < K) ? k0 + ORC_BLOCK : K;
+            float amax = 0.0f;
+            for (int k = k0; k < k1; ++k) {
+                float a = fabsf(bf16_to_f32(x[k]));
+                if (a > amax) amax = a;
+            }
+            const float s = block_scale(amax);
+            sfa[((size_t)g * KB + kb) * ld + m] = s;
+            for (int k = k0; k < k1; ++k) {
+                volatile float v = bf16_to_f32(x[k]) / s;   /* one fp32 division */
+                q[k] = oracle_e4m3_encode(v);
+            }
+        }
+    }
+}
+
+/* B side: X is [G][N][K] bf16, Q the codes, sfb the scales [G][ceil(N/128)][ceil(K/128)]. */
+void oracle_quantize_blocks(const uint16_t *X, int G, int N, int K, uint8_t *Q, float *sfb) {
+    const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
+    const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
+    long blocks = (long)G * NB * KB;
+    #pragma omp parallel for schedule(static)
+    for (long b = 0; b < blocks; ++b) {
+        const int g = (int)(b / ((long)NB * KB));
+        const int nb = (int)((b / KB) % NB), kb = (int)(b % KB);
+        const int n0 = nb * ORC_BLOCK, n1 = (n0 + ORC_BLOCK < N) ? n0 + ORC_BLOCK : N;
+        const int k0 = kb * ORC_BLOCK, k1 = (k0 + ORC_BLOCK < K) ? k0 + ORC_BLOCK : K;
+        const uint16_t *x = X + (size_t)g * N * K;
+        uint8_t *q = Q + (size_t)g * N * K;
+        float amax = 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int k = k0; k < k1; ++k) {
+                float a = fabsf(bf16_to_f32(x[(size_t)n * K + k]));
+                if (a > amax) amax = a;
+            }
+        const float s = block_scale(amax);
+        sfb[b] = s;
+        for (int n = n0; n < n1; ++n)
+            for (int k = k0; k < k1; ++k) {
+                volatile float v = bf16_to_f32(x[(size_t)n * K + k]) / s;
+                q[(size_t)n * K + k] = oracle_e4m3_encode(v);
+            }
     }
 }
 

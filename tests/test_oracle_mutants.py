@@ -70,3 +70,59 @@ def test_pins_catch_planted_mistake(name, tmp_path):
     finally:
         oracle._LIB = saved
     assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+# ---------------------------------------------------------------------------- the cast step
+from tests import test_oracle_cast as cast_pins  # noqa: E402
+
+CAST_MUTANTS = {
+    # ties rounded away from zero instead of to even
+    "cast_ties_away": ("else c = (lo % 2 == 0) ? lo : hi;", "else c = hi;"),
+    # the inverse scale
+    "cast_inverse_scale": ("volatile float s = amax / 448.0f;", "volatile float s = 448.0f / amax;"),
+    # non-saturating conversion: magnitudes above 448 become NaN
+    "cast_no_saturation": ("if (a >= dec[0x7E]) return sign | 0x7E;",
+                           "if (a > dec[0x7E]) return sign | 0x7F; if (a == dec[0x7E]) return sign | 0x7E;"),
+    # A scales stored row-major
+    "cast_sfa_row_major": ("sfa[((size_t)g * KB + kb) * ld + m] = s;", "sfa[((size_t)g * M + m) * KB + kb] = s;"),
+    # block maximum taken over the first row of the block only
+    "cast_block_amax_first_row": ("float a = fabsf(bf16_to_f32(x[(size_t)n * K + k]));",
+                                  "float a = (n == n0) ? fabsf(bf16_to_f32(x[(size_t)n * K + k])) : 0.0f;"),
+}
+
+CAST_PINS = [
+    cast_pins.test_encode_round_trips_every_finite_code,
+    cast_pins.test_encode_ties_to_even_and_neighbours,
+    cast_pins.test_encode_saturates,
+    cast_pins.test_encode_matches_torch_in_range,
+    cast_pins.test_hand_example_unit_scale,
+    lambda: cast_pins.test_rows_block_max_lands_on_448_and_rne_bound(7, 300),
+    cast_pins.test_rows_power_of_two_invariance_and_zero_block,
+    cast_pins.test_rows_scale_layout_column_major_and_grouped,
+    cast_pins.test_blocks_agree_with_rows_when_row_maxima_agree,
+    cast_pins.test_blocks_max_lands_on_448_per_block,
+    cast_pins.test_cast_then_gemm_approximates_the_bf16_product,
+]
+
+
+@pytest.mark.parametrize("name", sorted(CAST_MUTANTS))
+def test_cast_pins_catch_planted_mistake(name, tmp_path):
+    before, after = CAST_MUTANTS[name]
+    text = SRC.read_text()
+    assert text.count(before) == 1, name
+    (tmp_path / "m.c").write_text(text.replace(before, after))
+    so = tmp_path / f"liboracle_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC",
+                           "-shared", str(tmp_path / "m.c"), "-o", str(so), "-lm"])
+    saved = oracle._lib()
+    oracle._LIB = oracle.load(so)
+    caught = []
+    try:
+        for pin in CAST_PINS:
+            try:
+                pin()
+            except (AssertionError, ValueError, FloatingPointError):
+                caught.append(getattr(pin, "__name__", "rows_block_max"))
+    finally:
+        oracle._LIB = saved
+    assert caught, f"no pin caught the planted mistake {name!r}"
