@@ -41,6 +41,7 @@ L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_PER_BF16 = 2.0  # nominal dense fp8 / bf16 tensor throughput ratio (4.5 / 2.25 PFLOP/s)
 KERNEL_SOURCES = ["moe_grouped_gemm_08_b200/csrc/fp8_gemm_kernels.cuh",
+                  "moe_grouped_gemm_08_b200/csrc/fp8_cast_kernels.cuh",
                   "moe_grouped_gemm_08_b200/csrc/sm100_ptx.cuh",
                   "moe_grouped_gemm_08_b200/csrc/fp8gemm_api.cu"]
 
@@ -365,6 +366,74 @@ def run_reference(args, rank, world):
 METRIC = "FP8 TFLOPS & HBM GB/s per GEMM shape on 1xB200; % of FP8/HBM roofline"
 
 
+# ---------------------------------------------------------------------------- the cast step
+def run_cast(args, rank, world, local):
+    """Time the cast step (bf16 -> e4m3 + fp32 scales) on the prefill workload's operands: the
+    activations [4096, K] (1x128 row scales) and the weights [N, K] (128x128 block scales) of its
+    six GEMMs, 12 launches per step; about 1.1 GB moved per step, over 3x L2."""
+    import moe_grouped_gemm_08_b200 as fg
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = workloads.prefill()
+    g = torch.Generator(device=dev).manual_seed(5)
+    xs = [torch.randn((w["M"], w["K"]), generator=g, device=dev).to(torch.bfloat16) for w in wl]
+    ws = [torch.randn((w["N"], w["K"]), generator=g, device=dev).to(torch.bfloat16) for w in wl]
+    outs = [fg.cast_fp8_rows(x) for x in xs] + [fg.cast_fp8_blocks(w) for w in ws]
+
+    def launch_all():
+        s = torch.cuda.current_stream()
+        for x, (q, sfa) in zip(xs, outs[:len(xs)]):
+            fg._check(fg.lib.fp8_cast_rows(x.data_ptr(), q.data_ptr(), sfa.data_ptr(), 1, x.shape[0], x.shape[1],
+                                           fg._stream(s)), "cast rows")
+        for w, (q, sfb) in zip(ws, outs[len(xs):]):
+            fg._check(fg.lib.fp8_cast_blocks(w.data_ptr(), q.data_ptr(), sfb.data_ptr(), 1, w.shape[0], w.shape[1],
+                                             fg._stream(s)), "cast blocks")
+
+    def nbytes(M, K, rows):
+        kb = cdiv(K, 128)
+        return 3 * M * K + 4 * (M * kb if rows else cdiv(M, 128) * kb)
+    step_bytes = sum(nbytes(x.shape[0], x.shape[1], True) for x in xs) + \
+        sum(nbytes(w.shape[0], w.shape[1], False) for w in ws)
+    graph = torch.cuda.CUDAGraph()
+    launch_all()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        launch_all()
+    for _ in range(args.warmup):
+        graph.replay()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world, local)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
+    e0.record()
+    for _ in range(args.steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier(world, local)
+    clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    gbs = step_bytes * args.steps * world / (ms * 1e-3) / 1e9
+    peaks, peak_src = load_peaks()
+    del graph
+    if rank == 0:
+        line = {"metric": "HBM GB/s of the FP8 cast (bf16 -> e4m3 codes + fp32 scales)", "value": round(gbs, 1),
+                "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms / args.steps, 5), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16 -> e4m3", "data": "synthetic",
+                "config": {"workload": "cast_prefill_operands", "launches_per_step": 12,
+                           "bytes_per_step": step_bytes, "graph": "each step replayed from a CUDA graph"},
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                             "peak_source": f"{peak_src} (hbm_gbs)",
+                             "bytes_per_launch_def": "2 bytes read + 1 byte written per element + fp32 scales"},
+                "gpu_launches": 12 * args.steps, "clocks": clocks.summary(t0, t1)}
+        print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------- our arm
 def run_ours(args, rank, world, local):
     import moe_grouped_gemm_08_b200 as fg
@@ -562,7 +631,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--workload", default="decode_sweep",
-                    help="decode_sweep (default), dense_single, prefill, contiguous or masked")
+                    help="decode_sweep (default), dense_single, prefill, contiguous, masked, or cast (the bf16 -> "
+                         "e4m3 cast of the prefill operands)")
     ap.add_argument("--shape", default=None, help="M,N,K: one dense GEMM instead of a workload (profiling)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -582,6 +652,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "cast":
+            run_cast(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)
     finally:

@@ -132,6 +132,28 @@ fg_status fp8_gemm_nt_noalloc(const void* A, const float* sfa, const void* B, co
  * allocation-free variant (FG_OK if it was never called on this device). */
 fg_status fg_noalloc_status(void* stream);
 
+/* The cast step before the GEMM (the pages leave it to the user: turtlesai.it
+ * summary, FP8 casting and the TMA-aligned LHS scale layout are done outside the
+ * GEMM kernels).  X holds BF16 values; per block
+ *   scale = amax / 448 in fp32 (1 for an all-zero block),
+ *   code  = e4m3 round-to-nearest-even of the fp32 quotient x / scale, saturating
+ *           at +-448,
+ * so that dec(code) * scale approximates x.  Results are exact and deterministic
+ * (no accumulation).  K % 16 == 0; X and Q 16-byte aligned, scales 4-byte aligned;
+ * all pointers are device pointers owned by the caller; nothing is allocated.
+ *
+ * fp8_cast_rows: the A side (activations).  X is [G][M][K] (G = 1 for a plain
+ * [M, K] matrix), Q the e4m3 codes in the same layout, sfa one scale per 1 x 128
+ * block of a row in exactly the layout the GEMM entry points read:
+ * [G][ceil(K/128)][fg_sfa_ld(M)], column-major per group; its padding rows
+ * M .. ld-1 are not written.  G = 0 or M = 0 is a no-op. */
+fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K, void* stream);
+
+/* fp8_cast_blocks: the B side (weights).  X is [G][N][K], Q the codes, sfb one
+ * scale per 128 x 128 block: [G][ceil(N/128)][ceil(K/128)].  G = 0 or N = 0 is a
+ * no-op; G and ceil(N/128) must not exceed 65535. */
+fg_status fp8_cast_blocks(const void* X, void* Q, float* sfb, int G, int N, int K, void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word:
  * FG_OK, or FG_ERR_TIMEOUT if some kernel since the last call gave up a wait. */
 fg_status fg_get_device_status(void* stream);

@@ -44,6 +44,10 @@ _lib.fp8_gemm_grouped_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _in
 _lib.fp8_gemm_grouped_masked.restype = _int
 _lib.fp8_gemm_nt_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
 _lib.fp8_gemm_nt_noalloc.restype = _int
+_lib.fp8_cast_rows.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
+_lib.fp8_cast_rows.restype = _int
+_lib.fp8_cast_blocks.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
+_lib.fp8_cast_blocks.restype = _int
 _lib.fg_noalloc_status.argtypes = [_vp]
 _lib.fg_noalloc_status.restype = _int
 _lib.fg_get_device_status.argtypes = [_vp]
@@ -194,3 +198,37 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stre
                                         C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, _stream(stream)),
            "fp8_gemm_grouped_masked")
     return C
+
+
+# ---------------------------------------------------------------------------- the cast step
+def _bf16(t: torch.Tensor, what: str) -> torch.Tensor:
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{what} must be a contiguous CUDA bfloat16 tensor")
+    return t
+
+
+def cast_fp8_rows(x, stream=None):
+    """A side of the cast: x bf16 [M, K] or [G, M, K] -> (e4m3 codes as uint8, same shape;
+    sfa float32 [ceil(K/128), sfa_ld(M)] or [G, ceil(K/128), sfa_ld(M)]), one scale per 1 x 128
+    block of a row, in the column-major layout the GEMM entry points read."""
+    x = _bf16(x, "x")
+    grouped = x.dim() == 3
+    G, M, K = (x.shape if grouped else (1,) + tuple(x.shape))
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sfa = torch.zeros((G, _cdiv(K, 128), sfa_ld(M)), dtype=torch.float32, device=x.device)
+    _check(_lib.fp8_cast_rows(x.data_ptr(), q.data_ptr(), sfa.data_ptr(), G, M, K, _stream(stream)),
+           "fp8_cast_rows")
+    return q, (sfa if grouped else sfa[0])
+
+
+def cast_fp8_blocks(w, stream=None):
+    """B side of the cast: w bf16 [N, K] or [G, N, K] -> (e4m3 codes as uint8, same shape;
+    sfb float32 [ceil(N/128), ceil(K/128)] or [G, ...]), one scale per 128 x 128 block."""
+    w = _bf16(w, "w")
+    grouped = w.dim() == 3
+    G, N, K = (w.shape if grouped else (1,) + tuple(w.shape))
+    q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    sfb = torch.empty((G, _cdiv(N, 128), _cdiv(K, 128)), dtype=torch.float32, device=w.device)
+    _check(_lib.fp8_cast_blocks(w.data_ptr(), q.data_ptr(), sfb.data_ptr(), G, N, K, _stream(stream)),
+           "fp8_cast_blocks")
+    return q, (sfb if grouped else sfb[0])

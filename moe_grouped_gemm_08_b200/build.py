@@ -9,7 +9,8 @@ HERE = pathlib.Path(__file__).resolve().parent
 ROOT = HERE.parent
 SO = HERE / "libfp8gemm.so"
 SOURCES = [HERE / "csrc" / "fp8gemm_api.cu"]
-DEPENDS = SOURCES + [HERE / "csrc" / "fp8_gemm_kernels.cuh", HERE / "csrc" / "sm100_ptx.cuh",
+DEPENDS = SOURCES + [HERE / "csrc" / "fp8_gemm_kernels.cuh", HERE / "csrc" / "fp8_cast_kernels.cuh",
+                     HERE / "csrc" / "sm100_ptx.cuh",
                      ROOT / "include" / "fp8gemm.h"]
 
 NVCC_FLAGS = [

@@ -1,0 +1,117 @@
+// fp8_cast_kernels.cuh -- the cast step before the GEMM: BF16 values to e4m3 codes with
+// fine-grained fp32 scales, in the layouts the GEMM kernels read.
+//
+// The pages leave this step to the user (turtlesai.it summary: casting to FP8 and the transposed,
+// TMA-aligned LHS scales are done outside the GEMM library; news article: fine-grained scaling).
+// Per block -- 1 x 128 of a row of A, or 128 x 128 of B --
+//   scale = amax / 448 in fp32 (1 for an all-zero block), one IEEE division;
+//   code  = e4m3 round-to-nearest-even of the fp32 quotient x / scale, saturating at +-448.
+// Both kernels are bound by HBM: per element 2 bytes read and 1 byte written, plus one fp32
+// scale per 128 (rows) or 16384 (blocks) elements.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+namespace fg {
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& raw, float (&f)[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint2 encode_e4m3x8(const float (&f)[8], float scale) {
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    b[i] = static_cast<uint32_t>(__nv_cvt_float_to_fp8(__fdiv_rn(f[i], scale), __NV_SATFINITE, __NV_E4M3));
+  uint2 out;
+  out.x = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
+  out.y = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  return out;
+}
+
+__device__ __forceinline__ float cast_scale(float amax) { return amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f); }
+
+// A side.  X: bf16 [G*M][K] (row r = g*M + m), Q: e4m3 codes in the same layout, sfa:
+// [G][ceil(K/128)][ld], element (g, kb, m) at (g*KB + kb)*ld + m.  K % 8 == 0.
+// A warp takes one 256-column span of one row per step: lanes 0-15 the span's first K block,
+// lanes 16-31 its second; each lane 8 consecutive elements (one 16-byte load, one 8-byte store).
+__global__ void __launch_bounds__(256) fp8_cast_rows_kernel(const __nv_bfloat16* __restrict__ X,
+                                                            uint8_t* __restrict__ Q, float* __restrict__ sfa,
+                                                            int M, int K, int ld, long long rows, int spans) {
+  const int lane = threadIdx.x & 31;
+  const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  const int KB = (K + 127) / 128;
+  for (long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < rows * spans;
+       w += nwarps) {
+    const long long r = w / spans;
+    const int s = static_cast<int>(w - r * spans);
+    const int k = s * 256 + lane * 8;
+    const bool in = k < K;
+    float f[8];
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (in) raw = __ldg(reinterpret_cast<const uint4*>(X + r * K + k));
+    unpack_bf16x8(raw, f);
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));  // half-warp
+    const float scale = cast_scale(amax);
+    if (in) {
+      *reinterpret_cast<uint2*>(Q + r * K + k) = encode_e4m3x8(f, scale);
+      if ((lane & 15) == 0) {
+        const long long g = r / M;
+        const int m = static_cast<int>(r - g * M);
+        sfa[(g * KB + k / 128) * ld + m] = scale;
+      }
+    }
+  }
+}
+
+// B side.  X: bf16 [G][N][K], Q: codes, sfb: [G][ceil(N/128)][ceil(K/128)].  One CTA per 128 x 128
+// block (grid KB x NB x G): thread t holds rows t/16 + 16 i (i < 8) x columns 8 (t%16) .. +7 of
+// the block in registers, so the block is read once.  K % 8 == 0.
+__global__ void __launch_bounds__(256) fp8_cast_blocks_kernel(const __nv_bfloat16* __restrict__ X,
+                                                              uint8_t* __restrict__ Q, float* __restrict__ sfb,
+                                                              int N, int K) {
+  __shared__ float s_max[8];
+  const int kb = blockIdx.x, nb = blockIdx.y, g = blockIdx.z;
+  const int t = threadIdx.x;
+  const int k = kb * 128 + (t & 15) * 8;
+  const size_t base = static_cast<size_t>(g) * N * K;
+  float f[8][8];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = nb * 128 + (t >> 4) + 16 * i;
+    uint4 raw = make_uint4(0u, 0u, 0u, 0u);
+    if (n < N && k < K) raw = __ldg(reinterpret_cast<const uint4*>(X + base + static_cast<size_t>(n) * K + k));
+    unpack_bf16x8(raw, f[i]);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(f[i][j]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((t & 31) == 0) s_max[t >> 5] = amax;
+  __syncthreads();
+  amax = s_max[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, s_max[w]);
+  const float scale = cast_scale(amax);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int n = nb * 128 + (t >> 4) + 16 * i;
+    if (n < N && k < K)
+      *reinterpret_cast<uint2*>(Q + base + static_cast<size_t>(n) * K + k) = encode_e4m3x8(f[i], scale);
+  }
+  if (t == 0) sfb[(static_cast<size_t>(g) * gridDim.y + nb) * gridDim.x + kb] = scale;
+}
+
+}  // namespace fg

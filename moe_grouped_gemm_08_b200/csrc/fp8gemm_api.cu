@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "fp8_cast_kernels.cuh"
 #include "fp8_gemm_kernels.cuh"
 #include "fp8gemm.h"
 
@@ -585,6 +586,55 @@ fg_status fg_noalloc_status(void* stream) {
   if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FG_ERR_CUDA;
   if (v != 0 && cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
   return static_cast<fg_status>(v);
+}
+
+// ---------------------------------------------------------------------------- the cast step
+namespace {
+int sm_count_of_current() {
+  static std::atomic<int> cached[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) return 0;
+  cached[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+}  // namespace
+
+fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K, void* stream) {
+  if (!X || !Q || !sfa || G < 0 || M < 0 || K < 0) return FG_ERR_INVALID_ARG;
+  if (G == 0 || M == 0 || K == 0) return FG_OK;
+  if (K % 16 != 0 || !aligned(X, 16) || !aligned(Q, 16) || !aligned(sfa, 4)) return FG_ERR_ALIGNMENT;
+  if (static_cast<long long>(G) * M * K >= (1ll << 40)) return FG_ERR_UNSUPPORTED;
+  const int sms = sm_count_of_current();
+  if (sms <= 0) return FG_ERR_CUDA;
+  const long long rows = static_cast<long long>(G) * M;
+  const int spans = (K + 255) / 256;
+  const long long warps = rows * spans;
+  long long blocks = (warps + 7) / 8;
+  if (blocks > 8ll * sms) blocks = 8ll * sms;
+  // a plain (fully stream-ordered) launch: the kernel does not wait for a preceding grid itself
+  fg::fp8_cast_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(Q), sfa, M, K, fg_sfa_ld(M), rows, spans);
+  if (cudaGetLastError() != cudaSuccess) return FG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FG_OK;
+}
+
+fg_status fp8_cast_blocks(const void* X, void* Q, float* sfb, int G, int N, int K, void* stream) {
+  if (!X || !Q || !sfb || G < 0 || N < 0 || K < 0) return FG_ERR_INVALID_ARG;
+  if (G == 0 || N == 0 || K == 0) return FG_OK;
+  if (K % 16 != 0 || !aligned(X, 16) || !aligned(Q, 16) || !aligned(sfb, 4)) return FG_ERR_ALIGNMENT;
+  if (static_cast<long long>(G) * N * K >= (1ll << 40) || G > 65535 || (N + 127) / 128 > 65535)
+    return FG_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((N + 127) / 128),
+                  static_cast<unsigned>(G));
+  fg::fp8_cast_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(Q), sfb, N, K);
+  if (cudaGetLastError() != cudaSuccess) return FG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FG_OK;
 }
 
 fg_status fg_get_device_status(void* stream) {

@@ -78,3 +78,16 @@ def test_grouped_argument_errors():
     assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, P16, 2000, 64, 128, 128, NULL) == 3
     assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, P16, 2, 64, 128, 136, NULL) == 2
     assert L.fp8_gemm_grouped_masked(P16, P16, P16, P16, P16, P16, 0, 64, 128, 128, NULL) == 0
+
+
+def test_cast_argument_errors():
+    cast_rows, cast_blocks = fg.lib.fp8_cast_rows, fg.lib.fp8_cast_blocks
+    for f in (cast_rows, cast_blocks):
+        assert f(NULL, P16, P16, 1, 4, 128, NULL) == 1           # null input
+        assert f(P16, P16, P16, 1, 4, -128, NULL) == 1           # negative K
+        assert f(P16, P16, P16, 1, 4, 120, NULL) == 2            # K % 16
+        assert f(P16 + 8, P16, P16, 1, 4, 128, NULL) == 2        # X not 16-byte aligned
+        assert f(P16, P16 + 4, P16, 1, 4, 128, NULL) == 2        # Q not 16-byte aligned
+        assert f(P16, P16, P16, 0, 4, 128, NULL) == 0            # G = 0: no-op, nothing launched
+        assert f(P16, P16, P16, 1, 0, 128, NULL) == 0            # no rows: no-op
+    assert cast_blocks(P16, P16, P16, 70000, 4, 128, NULL) == 3  # more groups than a grid axis holds
