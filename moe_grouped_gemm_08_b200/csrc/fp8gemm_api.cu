@@ -610,13 +610,13 @@ fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K,
   const int sms = sm_count_of_current();
   if (sms <= 0) return FG_ERR_CUDA;
   const long long rows = static_cast<long long>(G) * M;
-  const int spans = (K + 255) / 256;
-  const long long warps = rows * spans;
+  const int chunks = (K + 256 * fg::kCastSpans - 1) / (256 * fg::kCastSpans);
+  const long long warps = rows * chunks;
   long long blocks = (warps + 7) / 8;
   if (blocks > 8ll * sms) blocks = 8ll * sms;
   // a plain (fully stream-ordered) launch: the kernel does not wait for a preceding grid itself
   fg::fp8_cast_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(Q), sfa, M, K, fg_sfa_ld(M), rows, spans);
+      static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(Q), sfa, M, K, fg_sfa_ld(M), rows, chunks);
   if (cudaGetLastError() != cudaSuccess) return FG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FG_OK;

@@ -101,3 +101,29 @@ def test_cast_then_gemm_on_gpu(fg):
     qa_ref, sfa_ref = oracle.quantize_rows(as_bits(x))
     qb_ref, sfb_ref = oracle.quantize_blocks(as_bits(w))
     close(bits_of(C), oracle.gemm_nt(qa_ref, sfa_ref, qb_ref, sfb_ref), "cast + gemm")
+
+
+@pytest.mark.parametrize("s", [1.5, 1.25, 1.75, 0.75])
+def test_cast_quotients_exactly_on_e4m3_midpoints(fg, s):
+    """With amax = 448 s the block scale is s; x = m * s (exact in bf16 for every e4m3 midpoint m)
+    makes x / s exactly a midpoint, a tie that x * RN(1/s) misses by an ulp: the kernel must still
+    round the exact quotient (to even), as the oracle does.  Neighbouring bf16 values included."""
+    d = oracle.e4m3_decode_table()
+    mids = (d[0:0x7E] + d[1:0x7F]) / 2
+    vals = np.concatenate([mids * s, np.nextafter(mids * s, np.inf), -mids * s]).astype(np.float32)
+    vals = torch.from_numpy(vals).to(torch.bfloat16).float().numpy()  # the neighbours become bf16 values
+    per_row = 127
+    nrows = (len(vals) + per_row - 1) // per_row
+    x = np.zeros((nrows, 128), dtype=np.float32)
+    x[:, 0] = 448.0 * s  # the block maximum fixes the scale at exactly s
+    flat = np.zeros(nrows * per_row, dtype=np.float32)
+    flat[:len(vals)] = vals
+    x[:, 1:] = flat.reshape(nrows, per_row)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    assert torch.equal(xb.float(), torch.from_numpy(x))  # every value is exact in bf16
+    q, sfa = fg.cast_fp8_rows(xb.cuda())
+    torch.cuda.synchronize()
+    q_ref, sfa_ref = oracle.quantize_rows(as_bits(xb))
+    assert np.all(sfa_ref[0, :nrows] == np.float32(s))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(sfa.cpu().numpy()[:, :nrows], sfa_ref[:, :nrows])
