@@ -4,7 +4,8 @@
  * The operation (all three entry points):
  *   C[m, n] = bf16( sum_kb  P_kb[m, n] * sfa[kb][m] * sfb[n / 128][kb] ),
  *   P_kb[m, n] = sum over the 128-wide K block kb of A[m, k] * B[n, k],
- * with A and B in FP8 e4m3, P_kb computed by the tensor cores and promoted into
+ * with A and B in FP8 (e4m3, or e5m2 through the _ex entry points), P_kb computed
+ * by the tensor cores and promoted into
  * FP32 accumulators once per K block ("two-level accumulation").
  * Sources:
  *   - "DeepGEMM" how-to (aisharenet.com), "Main functions" 1-3: the dense
@@ -65,6 +66,15 @@ typedef enum {
   FG_ERR_TIMEOUT = 6          /* a device-side wait ran out; the kernel exited early */
 } fg_status;
 
+/* FP8 operand formats (the aisharenet.com how-to, "Main functions": the FP8 inputs
+ * are E4M3 or E5M2).  The plain entry points take E4M3 for both operands; the _ex
+ * variants take each operand's format.  Scales are fp32 in the same layouts for
+ * both formats. */
+typedef enum {
+  FG_E4M3 = 0, /* 1 sign, 4 exponent (bias 7), 3 mantissa bits; largest finite 448 */
+  FG_E5M2 = 1  /* 1 sign, 5 exponent (bias 15), 2 mantissa bits; largest finite 57344 */
+} fg_fp8_format;
+
 /* Prepare the library on `device` (makes it current): queries the SM count,
  * resolves the tensor-map encoder and allocates the status word, the split-K
  * workspace and counters.  Idempotent.  Call it outside any stream capture. */
@@ -104,6 +114,18 @@ fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const voi
 fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb,
                                   void* C, const int* masked_m, int G, int Mmax, int N, int K,
                                   void* stream);
+
+/* The three GEMMs above with an explicit format for A (fmt_a) and for B (fmt_b):
+ * FG_E4M3 or FG_E5M2 each, mixed allowed; any other value is FG_ERR_INVALID_ARG.
+ * Everything else is as for the plain entry points. */
+fg_status fp8_gemm_nt_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                         int M, int N, int K, int fmt_a, int fmt_b, void* stream);
+fg_status fp8_gemm_grouped_contiguous_ex(const void* A, const float* sfa, const void* B, const float* sfb,
+                                         void* C, const int* m_indices, int M_total, int G, int N, int K,
+                                         int fmt_a, int fmt_b, void* stream);
+fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void* B, const float* sfb,
+                                     void* C, const int* masked_m, int G, int Mmax, int N, int K,
+                                     int fmt_a, int fmt_b, void* stream);
 
 /* Allocation-free variant of fp8_gemm_nt, for callers that cannot allocate device
  * memory: code running inside another framework's memory pool or a pre-planned

@@ -44,6 +44,13 @@ _lib.fp8_gemm_grouped_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _in
 _lib.fp8_gemm_grouped_masked.restype = _int
 _lib.fp8_gemm_nt_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
 _lib.fp8_gemm_nt_noalloc.restype = _int
+_lib.fp8_gemm_nt_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp]
+_lib.fp8_gemm_nt_ex.restype = _int
+_lib.fp8_gemm_grouped_contiguous_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
+                                                _vp]
+_lib.fp8_gemm_grouped_contiguous_ex.restype = _int
+_lib.fp8_gemm_grouped_masked_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _vp]
+_lib.fp8_gemm_grouped_masked_ex.restype = _int
 _lib.fp8_cast_rows.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
 _lib.fp8_cast_rows.restype = _int
 _lib.fp8_cast_blocks.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
@@ -110,14 +117,24 @@ def device_status(stream=None) -> int:
     return int(_lib.fg_get_device_status(ctypes.c_void_p(s.cuda_stream)))
 
 
-def _bytes(t: torch.Tensor, what: str) -> torch.Tensor:
+FORMATS = {"e4m3": 0, "e5m2": 1}
+
+
+def _bytes(t: torch.Tensor, what: str, fmt=None):
+    """FP8 operand -> (uint8 view, format code).  float8_e4m3fn / float8_e5m2 tensors carry their
+    format; uint8 codes are e4m3 unless ``fmt`` ("e4m3" or "e5m2") says otherwise."""
+    code = 0
     if t.dtype == torch.float8_e4m3fn:
         t = t.view(torch.uint8)
+    elif t.dtype == torch.float8_e5m2:
+        t, code = t.view(torch.uint8), 1
     if t.dtype != torch.uint8:
-        raise TypeError(f"{what} must be uint8 e4m3 codes or float8_e4m3fn, got {t.dtype}")
+        raise TypeError(f"{what} must be uint8 codes, float8_e4m3fn or float8_e5m2, got {t.dtype}")
+    if fmt is not None:
+        code = FORMATS[fmt]
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{what} must be a contiguous CUDA tensor")
-    return t
+    return t, code
 
 
 def _f32(t: torch.Tensor, what: str) -> torch.Tensor:
@@ -149,9 +166,10 @@ def _cdiv(a, b):
     return (a + b - 1) // b
 
 
-def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None):
-    """Dense C[M,N] = A[M,K] . B[N,K]^T with 1x128 (A) and 128x128 (B) fp32 scales."""
-    A, B = _bytes(A, "A"), _bytes(B, "B")
+def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=None):
+    """Dense C[M,N] = A[M,K] . B[N,K]^T with 1x128 (A) and 128x128 (B) fp32 scales; A and B are
+    e4m3 or e5m2 (from their dtype, or fmt_a / fmt_b for uint8 codes)."""
+    (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb = _f32(sfa, "sfa"), _f32(sfb, "sfb")
     M, K = A.shape
     N = B.shape[0]
@@ -160,14 +178,15 @@ def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None):
         raise ValueError("inconsistent shapes")
     C = _out(C, (M, N), A.device)
     init(A.device.index)
-    _check(_lib.fp8_gemm_nt(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
-                            M, N, K, _stream(stream)), "fp8_gemm_nt")
+    _check(_lib.fp8_gemm_nt_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
+                               M, N, K, fa, fb, _stream(stream)), "fp8_gemm_nt")
     return C
 
 
-def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None, stream=None):
+def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None, stream=None, fmt_a=None,
+                                              fmt_b=None):
     """M-grouped contiguous: A[M_total,K], B[G,N,K], m_indices[M_total] (-1 = padding)."""
-    A, B = _bytes(A, "A"), _bytes(B, "B")
+    (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb, m_indices = _f32(sfa, "sfa"), _f32(sfb, "sfb"), _i32(m_indices, "m_indices")
     M, K = A.shape
     G, N = B.shape[0], B.shape[1]
@@ -176,15 +195,15 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None,
         raise ValueError("inconsistent shapes")
     C = _out(C, (M, N), A.device)
     init(A.device.index)
-    _check(_lib.fp8_gemm_grouped_contiguous(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                            C.data_ptr(), m_indices.data_ptr(), M, G, N, K, _stream(stream)),
-           "fp8_gemm_grouped_contiguous")
+    _check(_lib.fp8_gemm_grouped_contiguous_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                               C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb,
+                                               _stream(stream)), "fp8_gemm_grouped_contiguous")
     return C
 
 
-def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stream=None):
+def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stream=None, fmt_a=None, fmt_b=None):
     """M-grouped masked: A[G,Mmax,K], masked_m[G] on the device; rows >= masked_m[g] untouched."""
-    A, B = _bytes(A, "A"), _bytes(B, "B")
+    (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb, masked_m = _f32(sfa, "sfa"), _f32(sfb, "sfb"), _i32(masked_m, "masked_m")
     G, Mmax, K = A.shape
     N = B.shape[1]
@@ -194,8 +213,8 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stre
         raise ValueError("inconsistent shapes")
     C = _out(C, (G, Mmax, N), A.device)
     init(A.device.index)
-    _check(_lib.fp8_gemm_grouped_masked(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                        C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, _stream(stream)),
+    _check(_lib.fp8_gemm_grouped_masked_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                           C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb, _stream(stream)),
            "fp8_gemm_grouped_masked")
     return C
 

@@ -76,6 +76,7 @@ struct TiledParams {
   int m_blocks; // ceil(M / 128)
   int n_blocks; // ceil(N / BN)
   int group_m;  // tile order: groups of group_m m-blocks, m-block fastest inside a group
+  uint32_t fmt_bits;  // operand formats in instruction-descriptor position (0: both e4m3)
 };
 
 struct SwapParams {
@@ -89,6 +90,7 @@ struct SwapParams {
   int num_kb;
   int n_tiles;     // ceil(N / 128)
   int debug_stall; // test hook: 1 = the MMA thread first waits on a barrier no one arrives at
+  uint32_t fmt_bits;  // operand formats in instruction-descriptor position (MMA A = weights)
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -370,7 +372,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           const uint64_t bdesc = smem_desc_k128_sw128(st + A_BYTES);
 #pragma unroll
           for (int j = 0; j < kBlockK / 32; ++j)  // 32 e4m3 = 32 bytes = 2 descriptor units per step
-            mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+            mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
           mma_commit(&empty[stage]);
           mma_commit(&tfull[tb]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -715,7 +717,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
             const uint64_t bdesc = smem_desc_k128_sw128(st + A_BYTES);
 #pragma unroll
             for (int j = 0; j < kBlockK / 32; ++j)
-              mma_f8_pair(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+              mma_f8_pair(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
             mma_commit_pair(&empty[stage], kBoth);
             mma_commit_pair(&tfull[tb], kBoth);
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -1020,7 +1022,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t bdesc = smem_desc_k128_sw128(sw + W_BYTES);
 #pragma unroll
         for (int j = 0; j < kBlockK / 32; ++j)
-          mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC, j > 0 ? 1u : 0u);
+          mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
         mma_commit(&empty[stage]);
         mma_commit(&tfull[tb]);
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }

@@ -204,10 +204,12 @@ fg_status check_common(const void* A, const float* sfa, const void* B, const flo
 
 template <int MODE>
 fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                    const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream) {
+                    const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
+                    int fmt_a, int fmt_b) {
   constexpr int BN = kTiledBN;
   constexpr int STAGES = kTiledStages;
   fg::TiledParams p;
+  p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
   p.sfa = sfa;
   p.sfb = sfb;
   p.C = static_cast<__nv_bfloat16*>(C);
@@ -279,12 +281,13 @@ int pair_capacity(int sms, size_t smem) {
 
 template <int MODE>
 fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                   const int* masked_m, int M, int G, int N, int K, cudaStream_t stream) {
+                   const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
   constexpr int BN = kPairBN;
   constexpr int STAGES = kPairStages;
   constexpr auto KERNEL = fg::fp8_gemm_pair_kernel<BN, STAGES, MODE>;
   constexpr size_t SMEM = pair_smem_bytes<BN, STAGES>();
   fg::TiledParams p;
+  p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
   p.sfa = sfa;
   p.sfb = sfb;
   p.C = static_cast<__nv_bfloat16*>(C);
@@ -326,9 +329,11 @@ fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void*
 
 template <int MP>
 fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                   int M, int N, int K, cudaStream_t stream) {
+                   int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
   constexpr int STAGES = swap_stages<MP>();
   fg::SwapParams p;
+  // swap-AB: the MMA's A operand is the weight tile (B of the GEMM), its B operand the tokens
+  p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_b), static_cast<uint32_t>(fmt_a));
   p.sfa = sfa;
   p.sfb = sfb;
   p.C = static_cast<__nv_bfloat16*>(C);
@@ -415,6 +420,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.num_kb = (K + kBlockK - 1) / kBlockK;
   p.n_tiles = (N + kBlockM - 1) / kBlockM;
   p.debug_stall = 0;
+  p.fmt_bits = 0;  // e4m3 x e4m3
   if (p.n_tiles > kNoAllocCounters) return FG_ERR_UNSUPPORTED;
   // the counters must start at zero; the kernel leaves them at zero, but a call that gave up a
   // wait may not have, so clear the ones this call uses (a memset, no allocation)
@@ -498,9 +504,13 @@ uint64_t fg_launch_count(void) { return g_launches.load(); }
 
 int fg_debug_set_stall(int enable) { return g_debug_stall.exchange(enable ? 1 : 0); }
 
-fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
-                      int K, void* stream) {
-  if (M < 0 || N < 0) return FG_ERR_INVALID_ARG;
+static bool valid_formats(int fmt_a, int fmt_b) {
+  return (fmt_a == FG_E4M3 || fmt_a == FG_E5M2) && (fmt_b == FG_E4M3 || fmt_b == FG_E5M2);
+}
+
+fg_status fp8_gemm_nt_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
+                         int K, int fmt_a, int fmt_b, void* stream) {
+  if (M < 0 || N < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return FG_OK;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
   if (s != FG_OK) return s;
@@ -513,17 +523,23 @@ fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const floa
   const bool swap = (path == 2) || (path == 0 && M <= kMaxSwapMP);
   if (swap) {
     if (M > kMaxSwapMP) return FG_ERR_UNSUPPORTED;
-    if (M <= 32) return run_swap<32>(st, A, sfa, B, sfb, C, M, N, K, cs);
-    if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs);
-    return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs);
+    if (M <= 32) return run_swap<32>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b);
+    if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b);
+    return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b);
   }
-  if (path == 3) return run_pair<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, M, 1, N, K, cs);
-  return run_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs);
+  if (path == 3) return run_pair<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
+  return run_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
 }
 
-fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                                      const int* m_indices, int M_total, int G, int N, int K, void* stream) {
-  if (M_total < 0 || N < 0 || G < 0) return FG_ERR_INVALID_ARG;
+fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
+                      int K, void* stream) {
+  return fp8_gemm_nt_ex(A, sfa, B, sfb, C, M, N, K, FG_E4M3, FG_E4M3, stream);
+}
+
+fg_status fp8_gemm_grouped_contiguous_ex(const void* A, const float* sfa, const void* B, const float* sfb,
+                                         void* C, const int* m_indices, int M_total, int G, int N, int K, int fmt_a,
+                                         int fmt_b, void* stream) {
+  if (M_total < 0 || N < 0 || G < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
   if (M_total == 0 || N == 0) return FG_OK;
   if (G == 0) return FG_ERR_INVALID_ARG;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
@@ -535,12 +551,18 @@ fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const voi
   DeviceState* st = state_for_current(&s);
   if (!st) return s;
   return run_tiled<fg::kContiguous>(st, A, sfa, B, sfb, C, m_indices, nullptr, M_total, G, N, K,
-                                    static_cast<cudaStream_t>(stream));
+                                    static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
 }
 
-fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                                  const int* masked_m, int G, int Mmax, int N, int K, void* stream) {
-  if (G < 0 || Mmax < 0 || N < 0) return FG_ERR_INVALID_ARG;
+fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                                      const int* m_indices, int M_total, int G, int N, int K, void* stream) {
+  return fp8_gemm_grouped_contiguous_ex(A, sfa, B, sfb, C, m_indices, M_total, G, N, K, FG_E4M3, FG_E4M3, stream);
+}
+
+fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                                     const int* masked_m, int G, int Mmax, int N, int K, int fmt_a, int fmt_b,
+                                     void* stream) {
+  if (G < 0 || Mmax < 0 || N < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
   if (G == 0 || Mmax == 0 || N == 0) return FG_OK;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
   if (s != FG_OK) return s;
@@ -552,9 +574,15 @@ fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B
   DeviceState* st = state_for_current(&s);
   if (!st) return s;
   if (g_dense_path.load() == 3)
-    return run_pair<fg::kMasked>(st, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K, static_cast<cudaStream_t>(stream));
+    return run_pair<fg::kMasked>(st, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K, static_cast<cudaStream_t>(stream),
+                                 fmt_a, fmt_b);
   return run_tiled<fg::kMasked>(st, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
-                                static_cast<cudaStream_t>(stream));
+                                static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
+}
+
+fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                                  const int* masked_m, int G, int Mmax, int N, int K, void* stream) {
+  return fp8_gemm_grouped_masked_ex(A, sfa, B, sfb, C, masked_m, G, Mmax, N, K, FG_E4M3, FG_E4M3, stream);
 }
 
 fg_status fp8_gemm_nt_noalloc(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M,

@@ -339,6 +339,12 @@ __device__ __forceinline__ uint64_t smem_desc_k128_sw128(uint32_t saddr) {
   return d;
 }
 
+// Operand-format field of the instruction descriptor (kind::f8f6f4): a at bits 7-9, b at 10-12;
+// 0 = e4m3, 1 = e5m2.
+__host__ __device__ constexpr uint32_t idesc_formats(uint32_t a_fmt, uint32_t b_fmt) {
+  return (a_fmt << 7) | (b_fmt << 10);
+}
+
 // Instruction descriptor: e4m3 x e4m3 -> f32, both operands K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4)                                  // D format: f32

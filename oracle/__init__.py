@@ -49,13 +49,14 @@ def load(path) -> ctypes.CDLL:
     lib.oracle_e4m3_decode_table.argtypes = [vp]
     lib.oracle_bf16_from_f64.restype = ctypes.c_uint16
     lib.oracle_bf16_from_f64.argtypes = [ctypes.c_double]
-    lib.oracle_gemm_nt.argtypes = [vp, vp, c_long, vp, vp, c_int, c_int, c_int, vp, vp]
+    lib.oracle_e5m2_decode_table.argtypes = [vp]
+    lib.oracle_gemm_nt.argtypes = [vp, vp, c_long, vp, vp, c_int, c_int, c_int, vp, vp, c_int, c_int]
     lib.oracle_gemm_nt_rows.argtypes = [vp, vp, c_long, vp, vp, c_int, c_int, c_int,
-                                        vp, c_int, vp, vp]
+                                        vp, c_int, vp, vp, c_int, c_int]
     lib.oracle_grouped_contiguous.argtypes = [vp, vp, c_long, vp, vp, vp, c_int, c_int,
-                                              c_int, c_int, vp, c_int, vp, vp]
+                                              c_int, c_int, vp, c_int, vp, vp, c_int, c_int]
     lib.oracle_grouped_masked.argtypes = [vp, vp, c_long, vp, vp, vp, c_int, c_int,
-                                          c_int, c_int, vp, vp]
+                                          c_int, c_int, vp, vp, c_int, c_int]
     lib.oracle_num_threads.restype = c_int
     lib.oracle_e4m3_encode_array.argtypes = [vp, c_long, vp]
     lib.oracle_quantize_rows.argtypes = [vp, c_int, c_int, c_int, vp, vp, c_long]
@@ -88,6 +89,12 @@ def e4m3_decode_table() -> np.ndarray:
     return out
 
 
+def e5m2_decode_table() -> np.ndarray:
+    out = np.empty(256, dtype=np.float64)
+    _lib().oracle_e5m2_decode_table(_p(out))
+    return out
+
+
 def bf16_from_f64(x: float) -> int:
     return int(_lib().oracle_bf16_from_f64(float(x)))
 
@@ -96,8 +103,16 @@ def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
     return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
-def gemm_nt(A, sfa, B, sfb, want_acc: bool = False, rows=None):
-    """Dense C = A . B^T.  A[M,K] e4m3 codes, sfa[KB, ld], B[N,K], sfb[NB, KB].
+FORMATS = {"e4m3": 0, "e5m2": 1}
+
+
+def _fmt(f) -> int:
+    return FORMATS[f] if isinstance(f, str) else int(f)
+
+
+def gemm_nt(A, sfa, B, sfb, want_acc: bool = False, rows=None, fmt_a="e4m3", fmt_b="e4m3"):
+    """Dense C = A . B^T.  A[M,K] fp8 codes (fmt_a: e4m3 or e5m2), sfa[KB, ld], B[N,K] (fmt_b),
+    sfb[NB, KB].
 
     Returns bf16 bit patterns (uint16 [M or len(rows), N]) and, if asked, the fp64
     values before the final rounding.
@@ -111,16 +126,18 @@ def gemm_nt(A, sfa, B, sfb, want_acc: bool = False, rows=None):
     C = np.zeros((nrows, N), dtype=np.uint16)
     acc = np.zeros((nrows, N), dtype=np.float64) if want_acc else None
     if rows is None:
-        _lib().oracle_gemm_nt(_p(A), _p(sfa), ld, _p(B), _p(sfb), M, N, K, _p(C), _p(acc))
+        _lib().oracle_gemm_nt(_p(A), _p(sfa), ld, _p(B), _p(sfb), M, N, K, _p(C), _p(acc),
+                              _fmt(fmt_a), _fmt(fmt_b))
     else:
         r = _c(rows, np.int32)
         assert r.size == 0 or (r.min() >= 0 and r.max() < M)
         _lib().oracle_gemm_nt_rows(_p(A), _p(sfa), ld, _p(B), _p(sfb), M, N, K,
-                                   _p(r), int(r.size), _p(C), _p(acc))
+                                   _p(r), int(r.size), _p(C), _p(acc), _fmt(fmt_a), _fmt(fmt_b))
     return (C, acc) if want_acc else C
 
 
-def grouped_contiguous(A, sfa, B, sfb, m_indices, C=None, rows=None, want_acc: bool = False):
+def grouped_contiguous(A, sfa, B, sfb, m_indices, C=None, rows=None, want_acc: bool = False,
+                       fmt_a="e4m3", fmt_b="e4m3"):
     """M-grouped contiguous: A[M_total,K], B[G,N,K], sfb[G,NB,KB], m_indices[M_total].
 
     Rows with m_indices == -1 are left as they are in ``C`` (zeros if C is None).
@@ -140,11 +157,12 @@ def grouped_contiguous(A, sfa, B, sfb, m_indices, C=None, rows=None, want_acc: b
     acc = np.zeros((nrows, N), dtype=np.float64) if want_acc else None
     r = None if rows is None else _c(rows, np.int32)
     _lib().oracle_grouped_contiguous(_p(A), _p(sfa), ld, _p(B), _p(sfb), _p(mi), M_total, G,
-                                     N, K, _p(r), 0 if r is None else int(r.size), _p(C), _p(acc))
+                                     N, K, _p(r), 0 if r is None else int(r.size), _p(C), _p(acc),
+                                     _fmt(fmt_a), _fmt(fmt_b))
     return (C, acc) if want_acc else C
 
 
-def grouped_masked(A, sfa, B, sfb, masked_m, C=None, want_acc: bool = False):
+def grouped_masked(A, sfa, B, sfb, masked_m, C=None, want_acc: bool = False, fmt_a="e4m3", fmt_b="e4m3"):
     """M-grouped masked: A[G,Mmax,K], sfa[G,KB,ld], B[G,N,K], sfb[G,NB,KB], masked_m[G].
 
     Rows at or past masked_m[g] keep their values from ``C`` (zeros if C is None).
@@ -161,7 +179,7 @@ def grouped_masked(A, sfa, B, sfb, masked_m, C=None, want_acc: bool = False):
         C = np.array(C, dtype=np.uint16, copy=True, order="C")
     acc = np.zeros((G, Mmax, N), dtype=np.float64) if want_acc else None
     _lib().oracle_grouped_masked(_p(A), _p(sfa), ld, _p(B), _p(sfb), _p(mm), G, Mmax, N, K,
-                                 _p(C), _p(acc))
+                                 _p(C), _p(acc), _fmt(fmt_a), _fmt(fmt_b))
     return (C, acc) if want_acc else C
 
 

@@ -19,6 +19,8 @@
  *   - DeepSeek DeepGEMM news article (senqingzn.com), optimisation paragraph:
  *     the FP8 tensor-core accumulation is not precise enough, so partial sums
  *     are promoted into a higher-precision accumulator.
+ * Operands are e4m3 codes by default; either operand may instead be e5m2
+ * (the how-to, "Main functions": E4M3 or E5M2 inputs).
  * The pages leave the scale granularities open.  This oracle takes 1x128
  * (one fp32 scale per row of A per 128-wide K block, stored column-major with
  * leading dimension ld) and 128x128 (one fp32 scale per 128x128 block of B).
@@ -75,6 +77,57 @@ static const double *dec_table(void) {
     return g_dec;
 }
 
+/* ---------------------------------------------------------------------------
+ * e5m2 decode table, from the format definition: 1 sign bit, 5 exponent bits
+ * with bias 15, 2 mantissa bits; exponent field 0 encodes subnormals
+ * m/4 * 2^-14; exponent field 31 encodes infinity (m = 0) and NaN.  The
+ * largest finite magnitude is 1.75 * 2^15 = 57344.  ("DeepGEMM" how-to,
+ * aisharenet.com, "Main functions": the FP8 inputs are E4M3 or E5M2.)
+ * ------------------------------------------------------------------------- */
+static double g_dec52[256];
+static int g_dec52_ready = 0;
+
+static void build_decode_table_e5m2(void) {
+    for (int code = 0; code < 256; ++code) {
+        int sign = (code >> 7) & 1;
+        int e = (code >> 2) & 0x1F;
+        int m = code & 0x3;
+        double v;
+        if (e == 0x1F) {
+            v = m == 0 ? INFINITY : NAN;
+        } else if (e == 0) {
+            v = ldexp((double)m / 4.0, -14);
+        } else {
+            v = ldexp(1.0 + (double)m / 4.0, e - 15);
+        }
+        g_dec52[code] = sign ? -v : v;
+    }
+    g_dec52_ready = 1;
+}
+
+/* fmt 0: e4m3, 1: e5m2 */
+static const double *dec_table_fmt(int fmt) {
+    if (fmt == 0) return dec_table();
+    if (!g_dec52_ready) build_decode_table_e5m2();
+    return g_dec52;
+}
+
+void oracle_e5m2_decode_table(double *out256) {
+    memcpy(out256, dec_table_fmt(1), 256 * sizeof(double));
+}
+
+/* Every finite code of a format is an integer multiple of the format's quantum:
+ * 2^-9 for e4m3, 2^-16 for e5m2.  Products of e5m2 codes span more than 53 bits,
+ * so K-block sums that involve e5m2 are formed exactly in 128-bit integers in
+ * these units and converted to fp64 once (one rounding, relative 2^-53). */
+static int quantum_exp(int fmt) { return fmt == 0 ? 9 : 16; }
+
+static int64_t code_units(int fmt, uint8_t code) {
+    double v = dec_table_fmt(fmt)[code];
+    if (!isfinite(v)) return 0;  /* inputs are finite */
+    return (int64_t)ldexp(v, quantum_exp(fmt));
+}
+
 void oracle_e4m3_decode_table(double *out256) {
     memcpy(out256, dec_table(), sizeof(double) * 256);
 }
@@ -113,9 +166,12 @@ uint16_t oracle_bf16_from_f64(double x) {
  * ------------------------------------------------------------------------- */
 static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
                    const uint8_t *B, const float *sfb, int N, int K,
-                   uint16_t *c_row, double *acc_row) {
+                   uint16_t *c_row, double *acc_row, int fa, int fb) {
     const double *dec = dec_table();
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
+    int64_t ua[256], ub[256];
+    if (fa != 0 || fb != 0)
+        for (int c = 0; c < 256; ++c) { ua[c] = code_units(fa, (uint8_t)c); ub[c] = code_units(fb, (uint8_t)c); }
     for (int n = 0; n < N; ++n) {
         const uint8_t *b_row = B + (size_t)n * K;
         double acc = 0.0;
@@ -123,7 +179,13 @@ static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
             int k0 = kb * ORC_BLOCK;
             int k1 = k0 + ORC_BLOCK < K ? k0 + ORC_BLOCK : K;
             double s = 0.0;
-            for (int k = k0; k < k1; ++k) s += dec[a_row[k]] * dec[b_row[k]];
+            if (fa == 0 && fb == 0) {
+                for (int k = k0; k < k1; ++k) s += dec[a_row[k]] * dec[b_row[k]];
+            } else {
+                __int128 t = 0;
+                for (int k = k0; k < k1; ++k) t += (__int128)ua[a_row[k]] * ub[b_row[k]];
+                s = ldexp((double)t, -(quantum_exp(fa) + quantum_exp(fb)));
+            }
             double scale = (double)sfa_m[(size_t)kb * ld] *
                            (double)sfb[(size_t)(n / ORC_BLOCK) * KB + kb];
             acc += s * scale;
@@ -137,11 +199,11 @@ static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
  * acc (optional, M x N fp64) receives the unrounded values. */
 void oracle_gemm_nt(const uint8_t *A, const float *sfa, long ld,
                     const uint8_t *B, const float *sfb,
-                    int M, int N, int K, uint16_t *C, double *acc) {
+                    int M, int N, int K, uint16_t *C, double *acc, int fa, int fb) {
     #pragma omp parallel for schedule(dynamic, 1)
     for (int m = 0; m < M; ++m)
         row_nt(A + (size_t)m * K, sfa + m, ld, B, sfb, N, K,
-               C + (size_t)m * N, acc ? acc + (size_t)m * N : NULL);
+               C + (size_t)m * N, acc ? acc + (size_t)m * N : NULL, fa, fb);
 }
 
 /* Dense, selected rows only: row rows[i] of the product goes to C[i,:].
@@ -149,13 +211,13 @@ void oracle_gemm_nt(const uint8_t *A, const float *sfa, long ld,
 void oracle_gemm_nt_rows(const uint8_t *A, const float *sfa, long ld,
                          const uint8_t *B, const float *sfb,
                          int M, int N, int K, const int *rows, int nrows,
-                         uint16_t *C, double *acc) {
+                         uint16_t *C, double *acc, int fa, int fb) {
     (void)M;
     #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < nrows; ++i) {
         int m = rows[i];
         row_nt(A + (size_t)m * K, sfa + m, ld, B, sfb, N, K,
-               C + (size_t)i * N, acc ? acc + (size_t)i * N : NULL);
+               C + (size_t)i * N, acc ? acc + (size_t)i * N : NULL, fa, fb);
     }
 }
 
@@ -170,7 +232,7 @@ void oracle_grouped_contiguous(const uint8_t *A, const float *sfa, long ld,
                                const uint8_t *B, const float *sfb,
                                const int *m_indices, int M_total, int G,
                                int N, int K, const int *rows, int nrows,
-                               uint16_t *C, double *acc) {
+                               uint16_t *C, double *acc, int fa, int fb) {
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
     int count = rows ? nrows : M_total;
@@ -181,7 +243,7 @@ void oracle_grouped_contiguous(const uint8_t *A, const float *sfa, long ld,
         if (g < 0 || g >= G) continue;
         row_nt(A + (size_t)m * K, sfa + m, ld,
                B + (size_t)g * N * K, sfb + (size_t)g * NB * KB, N, K,
-               C + (size_t)i * N, acc ? acc + (size_t)i * N : NULL);
+               C + (size_t)i * N, acc ? acc + (size_t)i * N : NULL, fa, fb);
     }
 }
 
@@ -192,7 +254,7 @@ void oracle_grouped_contiguous(const uint8_t *A, const float *sfa, long ld,
 void oracle_grouped_masked(const uint8_t *A, const float *sfa, long ld,
                            const uint8_t *B, const float *sfb,
                            const int *masked_m, int G, int Mmax, int N, int K,
-                           uint16_t *C, double *acc) {
+                           uint16_t *C, double *acc, int fa, int fb) {
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
     long total = (long)G * Mmax;
@@ -206,7 +268,7 @@ void oracle_grouped_masked(const uint8_t *A, const float *sfa, long ld,
         row_nt(A + ((size_t)g * Mmax + m) * K, sfa + (size_t)g * KB * ld + m, ld,
                B + (size_t)g * N * K, sfb + (size_t)g * NB * KB, N, K,
                C + ((size_t)g * Mmax + m) * N,
-               acc ? acc + ((size_t)g * Mmax + m) * N : NULL);
+               acc ? acc + ((size_t)g * Mmax + m) * N : NULL, fa, fb);
     }
 }
 

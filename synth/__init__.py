@@ -58,7 +58,9 @@ def _lib():
         lib.synth_e4m3_encode.argtypes = [ctypes.c_float]
         lib.synth_quantize_1x128.argtypes = [vp, i64, c_int, vp, vp, i64]
         lib.synth_quantize_128x128.argtypes = [vp, i64, c_int, vp, vp]
-        lib.synth_quantized_matrix.argtypes = [u64, u64, i64, c_int, vp, c_int, vp, vp, i64]
+        lib.synth_e5m2_encode.restype = ctypes.c_uint8
+        lib.synth_e5m2_encode.argtypes = [ctypes.c_float]
+        lib.synth_quantized_matrix.argtypes = [u64, u64, i64, c_int, vp, c_int, vp, vp, i64, c_int]
         _LIB = lib
     return _LIB
 
@@ -113,22 +115,30 @@ def quantize_128x128(x: np.ndarray):
     return q, sf
 
 
+FORMATS = {"e4m3": 0, "e5m2": 1}
+
+
+def e5m2_encode(x: float) -> int:
+    return int(_lib().synth_e5m2_encode(float(x)))
+
+
 def quantized_a(stream: int, rows: int, K: int, ld: int | None = None,
-                row_scale: np.ndarray | None = None, offset: int = 0):
-    """Generate and quantise an A operand (1x128 blocks, column-major scales)."""
+                row_scale: np.ndarray | None = None, offset: int = 0, fmt: str = "e4m3"):
+    """Generate and quantise an A operand (1x128 blocks, column-major scales); fmt e4m3 or e5m2
+    (scale = amax / 448 or amax / 57344)."""
     ld = sfa_ld(rows) if ld is None else ld
     q = np.empty((rows, K), dtype=np.uint8)
     sf = np.zeros((cdiv(K, BLOCK), ld), dtype=np.float32)
     rs = None if row_scale is None else np.ascontiguousarray(row_scale, dtype=np.float32)
-    _lib().synth_quantized_matrix(stream, offset, rows, K, _ptr(rs), 0, _ptr(q), _ptr(sf), ld)
+    _lib().synth_quantized_matrix(stream, offset, rows, K, _ptr(rs), 0, _ptr(q), _ptr(sf), ld, FORMATS[fmt])
     return q, sf
 
 
-def quantized_b(stream: int, rows: int, K: int, offset: int = 0):
-    """Generate and quantise a B operand (128x128 blocks)."""
+def quantized_b(stream: int, rows: int, K: int, offset: int = 0, fmt: str = "e4m3"):
+    """Generate and quantise a B operand (128x128 blocks); fmt e4m3 or e5m2."""
     q = np.empty((rows, K), dtype=np.uint8)
     sf = np.empty((cdiv(rows, BLOCK), cdiv(K, BLOCK)), dtype=np.float32)
-    _lib().synth_quantized_matrix(stream, offset, rows, K, None, 1, _ptr(q), _ptr(sf), 0)
+    _lib().synth_quantized_matrix(stream, offset, rows, K, None, 1, _ptr(q), _ptr(sf), 0, FORMATS[fmt])
     return q, sf
 
 
@@ -138,26 +148,29 @@ def row_factors(seed: int, rows: int) -> np.ndarray:
     return (10.0 ** (4.0 * u - 2.0)).astype(np.float32)
 
 
-def dense_case(seed: int, M: int, N: int, K: int, row_scaled: bool = False) -> dict:
-    """Dense workload: A[M,K], sfa[KB, ld], B[N,K], sfb[NB, KB]."""
+def dense_case(seed: int, M: int, N: int, K: int, row_scaled: bool = False, fmt_a: str = "e4m3",
+               fmt_b: str = "e4m3") -> dict:
+    """Dense workload: A[M,K], sfa[KB, ld], B[N,K], sfb[NB, KB]; operands in e4m3 or e5m2."""
     rs = row_factors(seed, M) if row_scaled else None
-    A, sfa = quantized_a(2 * seed, M, K, row_scale=rs)
-    B, sfb = quantized_b(2 * seed + 1, N, K)
-    return dict(kind="dense", A=A, sfa=sfa, B=B, sfb=sfb, M=M, N=N, K=K, ld=sfa.shape[1])
+    A, sfa = quantized_a(2 * seed, M, K, row_scale=rs, fmt=fmt_a)
+    B, sfb = quantized_b(2 * seed + 1, N, K, fmt=fmt_b)
+    return dict(kind="dense", A=A, sfa=sfa, B=B, sfb=sfb, M=M, N=N, K=K, ld=sfa.shape[1], fmt_a=fmt_a,
+                fmt_b=fmt_b)
 
 
-def grouped_b(seed: int, G: int, N: int, K: int):
+def grouped_b(seed: int, G: int, N: int, K: int, fmt: str = "e4m3"):
     """B[G,N,K] with independent draws per expert; sfb[G, NB, KB]."""
     B = np.empty((G, N, K), dtype=np.uint8)
     sfb = np.empty((G, cdiv(N, BLOCK), cdiv(K, BLOCK)), dtype=np.float32)
     for g in range(G):
-        q, sf = quantized_b(2 * seed + 1, N, K, offset=g * N * K)
+        q, sf = quantized_b(2 * seed + 1, N, K, offset=g * N * K, fmt=fmt)
         B[g] = q
         sfb[g] = sf
     return B, sfb
 
 
-def contiguous_case(seed: int, group_rows, N: int, K: int, align: int = BLOCK) -> dict:
+def contiguous_case(seed: int, group_rows, N: int, K: int, align: int = BLOCK, fmt_a: str = "e4m3",
+                    fmt_b: str = "e4m3") -> dict:
     """M-grouped contiguous workload.
 
     group_rows[g] valid rows of expert g; each group is padded up to a multiple of
@@ -171,8 +184,8 @@ def contiguous_case(seed: int, group_rows, N: int, K: int, align: int = BLOCK) -
     for g, (r, p) in enumerate(zip(group_rows, padded)):
         m_indices[start:start + r] = g
         start += p
-    A, sfa = quantized_a(2 * seed, M_total, K)
-    B, sfb = grouped_b(seed, G, N, K)
+    A, sfa = quantized_a(2 * seed, M_total, K, fmt=fmt_a)
+    B, sfb = grouped_b(seed, G, N, K, fmt=fmt_b)
     return dict(kind="contiguous", A=A, sfa=sfa, B=B, sfb=sfb, m_indices=m_indices,
                 M=M_total, G=G, N=N, K=K, ld=sfa.shape[1], group_rows=list(group_rows))
 
@@ -188,17 +201,18 @@ def masked_counts(seed: int, G: int, Mmax: int) -> np.ndarray:
     return m
 
 
-def masked_case(seed: int, G: int, Mmax: int, N: int, K: int, masked_m=None) -> dict:
+def masked_case(seed: int, G: int, Mmax: int, N: int, K: int, masked_m=None, fmt_a: str = "e4m3",
+                fmt_b: str = "e4m3") -> dict:
     """M-grouped masked workload: A[G,Mmax,K], sfa[G,KB,ld], B[G,N,K], sfb[G,NB,KB]."""
     ld = sfa_ld(Mmax)
     KB = cdiv(K, BLOCK)
     A = np.empty((G, Mmax, K), dtype=np.uint8)
     sfa = np.zeros((G, KB, ld), dtype=np.float32)
     for g in range(G):
-        q, sf = quantized_a(2 * seed, Mmax, K, ld=ld, offset=g * Mmax * K)
+        q, sf = quantized_a(2 * seed, Mmax, K, ld=ld, offset=g * Mmax * K, fmt=fmt_a)
         A[g] = q
         sfa[g] = sf
-    B, sfb = grouped_b(seed, G, N, K)
+    B, sfb = grouped_b(seed, G, N, K, fmt=fmt_b)
     mm = masked_counts(seed, G, Mmax) if masked_m is None else np.asarray(masked_m, dtype=np.int32)
     return dict(kind="masked", A=A, sfa=sfa, B=B, sfb=sfb, masked_m=mm,
                 G=G, Mmax=Mmax, N=N, K=K, ld=ld)

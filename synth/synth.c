@@ -97,8 +97,50 @@ uint8_t synth_e4m3_encode(float xf) {
     return sign | code;
 }
 
+/* e5m2 encoder with round-to-nearest-even and saturation to +-57344.
+ * Written from the format: 2 mantissa bits, exponent bias 15, subnormal quantum
+ * 2^-16, largest finite 57344 = 1.75 * 2^15 (code 0x7B; 0x7C is infinity).
+ * NaN input maps to a NaN code (never produced by the generator). */
+uint8_t synth_e5m2_encode(float xf) {
+    double x = (double)xf;
+    if (isnan(x)) return 0x7E;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 57344.0) return sign | 0x7B;        /* saturate (also +-inf) */
+    if (a == 0.0) return sign;
+    int e;
+    (void)frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+    int q = e - 3;                      /* quantum for 3 significant bits */
+    if (q < -16) q = -16;               /* subnormal quantum */
+    double r = nearbyint(ldexp(a, -q)); /* ties to even */
+    double y = ldexp(r, q);
+    if (y > 57344.0) y = 57344.0;
+    if (y == 0.0) return sign;
+    int ey;
+    double fy = frexp(y, &ey);          /* y = fy * 2^ey, fy in [0.5, 1) */
+    int biased = ey - 1 + 15;
+    uint8_t code;
+    if (biased <= 0) {                  /* subnormal: y = m/4 * 2^-14 = m * 2^-16 */
+        code = (uint8_t)(int)ldexp(y, 16);
+    } else {
+        int m = (int)((fy * 2.0 - 1.0) * 4.0);
+        code = (uint8_t)((biased << 2) | m);
+    }
+    return sign | code;
+}
+
+/* fmt 0: e4m3 (largest finite 448), 1: e5m2 (largest finite 57344) */
+static inline uint8_t encode_fmt(float v, int fmt) {
+    return fmt == 0 ? synth_e4m3_encode(v) : synth_e5m2_encode(v);
+}
+
+static inline float block_scale_fmt(float amax, int fmt) {
+    const float top = fmt == 0 ? 448.0f : 57344.0f;
+    return amax > 0.0f ? amax / top : 1.0f;
+}
+
 static inline float block_scale(float amax) {
-    return amax > 0.0f ? amax / 448.0f : 1.0f;
+    return block_scale_fmt(amax, 0);
 }
 
 /* Quantise rows x[rows][K] (fp32) with 1x128 blocks.
@@ -147,7 +189,7 @@ void synth_quantize_128x128(const float *x, long rows, int K, uint8_t *q, float 
  * mode 1: 128x128 blocks, sf[rb][kb] (B operand). */
 void synth_quantized_matrix(uint64_t stream, uint64_t offset, long rows, int K,
                             const float *row_scale, int mode,
-                            uint8_t *q, float *sf, long ld) {
+                            uint8_t *q, float *sf, long ld, int fmt) {
     const int KB = (K + SY_BLOCK - 1) / SY_BLOCK;
     uint64_t key = stream_key(stream);
     if (mode == 0) {
@@ -166,8 +208,8 @@ void synth_quantized_matrix(uint64_t stream, uint64_t offset, long rows, int K,
                         buf[k - k0] = v;
                         float a = fabsf(v); if (a > amax) amax = a;
                     }
-                    float s = block_scale(amax);
-                    for (int k = k0; k < k1; ++k) q[r * K + k] = synth_e4m3_encode(buf[k - k0] / s);
+                    float s = block_scale_fmt(amax, fmt);
+                    for (int k = k0; k < k1; ++k) q[r * K + k] = encode_fmt(buf[k - k0] / s, fmt);
                     sf[(long)kb * ld + r] = s;
                 }
             }
@@ -192,10 +234,10 @@ void synth_quantized_matrix(uint64_t stream, uint64_t offset, long rows, int K,
                             float a = fabsf(v); if (a > amax) amax = a;
                         }
                     }
-                    float s = block_scale(amax);
+                    float s = block_scale_fmt(amax, fmt);
                     for (long r = r0; r < r1; ++r)
                         for (int k = k0; k < k1; ++k)
-                            q[r * K + k] = synth_e4m3_encode(tile[(r - r0) * SY_BLOCK + (k - k0)] / s);
+                            q[r * K + k] = encode_fmt(tile[(r - r0) * SY_BLOCK + (k - k0)] / s, fmt);
                     sf[rb * KB + kb] = s;
                 }
             }

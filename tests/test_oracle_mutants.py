@@ -126,3 +126,49 @@ def test_cast_pins_catch_planted_mistake(name, tmp_path):
     finally:
         oracle._LIB = saved
     assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+# ---------------------------------------------------------------------------- e5m2 operands
+from tests import test_oracle_e5m2 as e5m2_pins  # noqa: E402
+
+E5M2_MUTANTS = {
+    # exponent bias 16 instead of 15
+    "e5m2_bias": ("v = ldexp(1.0 + (double)m / 4.0, e - 15);", "v = ldexp(1.0 + (double)m / 4.0, e - 16);"),
+    # integer units of e5m2 off by one binade
+    "e5m2_quantum": ("return fmt == 0 ? 9 : 16;", "return fmt == 0 ? 9 : 15;"),
+    # the two operands' formats swapped
+    "e5m2_swapped": ("ua[c] = code_units(fa, (uint8_t)c); ub[c] = code_units(fb, (uint8_t)c);",
+                     "ua[c] = code_units(fb, (uint8_t)c); ub[c] = code_units(fa, (uint8_t)c);"),
+}
+
+E5M2_PINS = [
+    e5m2_pins.test_e5m2_table_matches_formula_and_torch,
+    lambda: [e5m2_pins.test_e5m2_brute_force(fa, fb, 3, 4, 32, 1)
+             for fa, fb in [("e5m2", "e5m2"), ("e4m3", "e5m2"), ("e5m2", "e4m3")]],
+    e5m2_pins.test_e5m2_extreme_codes_need_more_than_fp64,
+    e5m2_pins.test_e5m2_identity_gives_transpose,
+    e5m2_pins.test_mixed_formats_transpose_symmetry,
+]
+
+
+@pytest.mark.parametrize("name", sorted(E5M2_MUTANTS))
+def test_e5m2_pins_catch_planted_mistake(name, tmp_path):
+    before, after = E5M2_MUTANTS[name]
+    text = SRC.read_text()
+    assert text.count(before) == 1, name
+    (tmp_path / "m.c").write_text(text.replace(before, after))
+    so = tmp_path / f"liboracle_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC",
+                           "-shared", str(tmp_path / "m.c"), "-o", str(so), "-lm"])
+    saved = oracle._lib()
+    oracle._LIB = oracle.load(so)
+    caught = []
+    try:
+        for pin in E5M2_PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught.append(getattr(pin, "__name__", "brute_force"))
+    finally:
+        oracle._LIB = saved
+    assert caught, f"no pin caught the planted mistake {name!r}"

@@ -1,5 +1,6 @@
 """Checks of the seeded input generator (no GEMM arithmetic here)."""
 import numpy as np
+import torch
 
 import oracle
 import synth
@@ -70,3 +71,22 @@ def test_contiguous_layout_padding():
     assert (mi[:5] == 0).all() and (mi[5:128] == -1).all()
     assert (mi[128:258] == 1).all() and (mi[258:384] == -1).all()
     assert (mi[384:] == 3).all()
+
+
+def test_e5m2_encoder_matches_torch_in_range():
+    rng = np.random.default_rng(8)
+    v = np.concatenate([rng.uniform(-57344, 57344, 20000), rng.standard_normal(20000) * 1e-3,
+                        rng.standard_normal(20000)]).astype(np.float32)
+    mine = np.array([synth.e5m2_encode(x) for x in v], np.uint8)
+    ref = torch.from_numpy(v).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(mine, ref)
+    assert synth.e5m2_encode(1e9) == 0x7B and synth.e5m2_encode(-1e9) == 0xFB  # saturation at 57344
+
+
+def test_e5m2_operands_dequantise_close_to_the_draws():
+    c = synth.dense_case(3, 8, 130, 256, fmt_a="e5m2", fmt_b="e5m2")
+    dec = torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).double().numpy()
+    a = dec[c["A"]] * np.repeat(c["sfa"][:, :8].T, 128, axis=1)
+    assert np.all(np.abs(a).max(axis=1) > 0) and np.isfinite(a).all()
+    # the block maximum lands on the largest finite e5m2 value
+    assert np.all((c["A"][:, :128] & 0x7F).max(axis=1) == 0x7B)
