@@ -176,6 +176,12 @@ fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K,
  * no-op; G and ceil(N/128) must not exceed 65535. */
 fg_status fp8_cast_blocks(const void* X, void* Q, float* sfb, int G, int N, int K, void* stream);
 
+/* The two casts with a target format: FG_E4M3 (top = 448, as above) or FG_E5M2
+ * (scale = amax / 57344, codes saturating at +-57344); any other value is
+ * FG_ERR_INVALID_ARG. */
+fg_status fp8_cast_rows_ex(const void* X, void* Q, float* sfa, int G, int M, int K, int fmt, void* stream);
+fg_status fp8_cast_blocks_ex(const void* X, void* Q, float* sfb, int G, int N, int K, int fmt, void* stream);
+
 /* Synchronise `stream`, then read and clear the device status word:
  * FG_OK, or FG_ERR_TIMEOUT if some kernel since the last call gave up a wait. */
 fg_status fg_get_device_status(void* stream);

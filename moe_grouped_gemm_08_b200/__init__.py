@@ -55,6 +55,10 @@ _lib.fp8_cast_rows.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
 _lib.fp8_cast_rows.restype = _int
 _lib.fp8_cast_blocks.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
 _lib.fp8_cast_blocks.restype = _int
+_lib.fp8_cast_rows_ex.argtypes = [_vp, _vp, _vp, _int, _int, _int, _int, _vp]
+_lib.fp8_cast_rows_ex.restype = _int
+_lib.fp8_cast_blocks_ex.argtypes = [_vp, _vp, _vp, _int, _int, _int, _int, _vp]
+_lib.fp8_cast_blocks_ex.restype = _int
 _lib.fg_noalloc_status.argtypes = [_vp]
 _lib.fg_noalloc_status.restype = _int
 _lib.fg_get_device_status.argtypes = [_vp]
@@ -226,21 +230,21 @@ def _bf16(t: torch.Tensor, what: str) -> torch.Tensor:
     return t
 
 
-def cast_fp8_rows(x, stream=None):
+def cast_fp8_rows(x, stream=None, fmt="e4m3"):
     """A side of the cast: x bf16 [M, K] or [G, M, K] -> (e4m3 codes as uint8, same shape;
     sfa float32 [ceil(K/128), sfa_ld(M)] or [G, ceil(K/128), sfa_ld(M)]), one scale per 1 x 128
-    block of a row, in the column-major layout the GEMM entry points read."""
+    block of a row, in the column-major layout the GEMM entry points read; fmt "e4m3" or "e5m2"."""
     x = _bf16(x, "x")
     grouped = x.dim() == 3
     G, M, K = (x.shape if grouped else (1,) + tuple(x.shape))
     q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     sfa = torch.zeros((G, _cdiv(K, 128), sfa_ld(M)), dtype=torch.float32, device=x.device)
-    _check(_lib.fp8_cast_rows(x.data_ptr(), q.data_ptr(), sfa.data_ptr(), G, M, K, _stream(stream)),
-           "fp8_cast_rows")
+    _check(_lib.fp8_cast_rows_ex(x.data_ptr(), q.data_ptr(), sfa.data_ptr(), G, M, K, FORMATS[fmt],
+                                 _stream(stream)), "fp8_cast_rows")
     return q, (sfa if grouped else sfa[0])
 
 
-def cast_fp8_blocks(w, stream=None):
+def cast_fp8_blocks(w, stream=None, fmt="e4m3"):
     """B side of the cast: w bf16 [N, K] or [G, N, K] -> (e4m3 codes as uint8, same shape;
     sfb float32 [ceil(N/128), ceil(K/128)] or [G, ...]), one scale per 128 x 128 block."""
     w = _bf16(w, "w")
@@ -248,6 +252,6 @@ def cast_fp8_blocks(w, stream=None):
     G, N, K = (w.shape if grouped else (1,) + tuple(w.shape))
     q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
     sfb = torch.empty((G, _cdiv(N, 128), _cdiv(K, 128)), dtype=torch.float32, device=w.device)
-    _check(_lib.fp8_cast_blocks(w.data_ptr(), q.data_ptr(), sfb.data_ptr(), G, N, K, _stream(stream)),
-           "fp8_cast_blocks")
+    _check(_lib.fp8_cast_blocks_ex(w.data_ptr(), q.data_ptr(), sfb.data_ptr(), G, N, K, FORMATS[fmt],
+                                   _stream(stream)), "fp8_cast_blocks")
     return q, (sfb if grouped else sfb[0])

@@ -630,8 +630,8 @@ int sm_count_of_current() {
 }
 }  // namespace
 
-fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K, void* stream) {
-  if (!X || !Q || !sfa || G < 0 || M < 0 || K < 0) return FG_ERR_INVALID_ARG;
+fg_status fp8_cast_rows_ex(const void* X, void* Q, float* sfa, int G, int M, int K, int fmt, void* stream) {
+  if (!X || !Q || !sfa || G < 0 || M < 0 || K < 0 || (fmt != FG_E4M3 && fmt != FG_E5M2)) return FG_ERR_INVALID_ARG;
   if (G == 0 || M == 0 || K == 0) return FG_OK;
   if (K % 16 != 0 || !aligned(X, 16) || !aligned(Q, 16) || !aligned(sfa, 4)) return FG_ERR_ALIGNMENT;
   if (static_cast<long long>(G) * M * K >= (1ll << 40)) return FG_ERR_UNSUPPORTED;
@@ -643,26 +643,36 @@ fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K,
   long long blocks = (warps + 7) / 8;
   if (blocks > 8ll * sms) blocks = 8ll * sms;
   // a plain (fully stream-ordered) launch: the kernel does not wait for a preceding grid itself
-  fg::fp8_cast_rows_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  const auto kernel = fmt == FG_E4M3 ? fg::fp8_cast_rows_kernel<0> : fg::fp8_cast_rows_kernel<1>;
+  kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(Q), sfa, M, K, fg_sfa_ld(M), rows, chunks);
   if (cudaGetLastError() != cudaSuccess) return FG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FG_OK;
 }
 
-fg_status fp8_cast_blocks(const void* X, void* Q, float* sfb, int G, int N, int K, void* stream) {
-  if (!X || !Q || !sfb || G < 0 || N < 0 || K < 0) return FG_ERR_INVALID_ARG;
+fg_status fp8_cast_rows(const void* X, void* Q, float* sfa, int G, int M, int K, void* stream) {
+  return fp8_cast_rows_ex(X, Q, sfa, G, M, K, FG_E4M3, stream);
+}
+
+fg_status fp8_cast_blocks_ex(const void* X, void* Q, float* sfb, int G, int N, int K, int fmt, void* stream) {
+  if (!X || !Q || !sfb || G < 0 || N < 0 || K < 0 || (fmt != FG_E4M3 && fmt != FG_E5M2)) return FG_ERR_INVALID_ARG;
   if (G == 0 || N == 0 || K == 0) return FG_OK;
   if (K % 16 != 0 || !aligned(X, 16) || !aligned(Q, 16) || !aligned(sfb, 4)) return FG_ERR_ALIGNMENT;
   if (static_cast<long long>(G) * N * K >= (1ll << 40) || G > 65535 || (N + 127) / 128 > 65535)
     return FG_ERR_UNSUPPORTED;
   const dim3 grid(static_cast<unsigned>((K + 127) / 128), static_cast<unsigned>((N + 127) / 128),
                   static_cast<unsigned>(G));
-  fg::fp8_cast_blocks_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(Q), sfb, N, K);
+  const auto kernel = fmt == FG_E4M3 ? fg::fp8_cast_blocks_kernel<0> : fg::fp8_cast_blocks_kernel<1>;
+  kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<const __nv_bfloat16*>(X),
+                                                              static_cast<uint8_t*>(Q), sfb, N, K);
   if (cudaGetLastError() != cudaSuccess) return FG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
   return FG_OK;
+}
+
+fg_status fp8_cast_blocks(const void* X, void* Q, float* sfb, int G, int N, int K, void* stream) {
+  return fp8_cast_blocks_ex(X, Q, sfb, G, N, K, FG_E4M3, stream);
 }
 
 fg_status fg_get_device_status(void* stream) {

@@ -59,8 +59,9 @@ def load(path) -> ctypes.CDLL:
                                           c_int, c_int, vp, vp, c_int, c_int]
     lib.oracle_num_threads.restype = c_int
     lib.oracle_e4m3_encode_array.argtypes = [vp, c_long, vp]
-    lib.oracle_quantize_rows.argtypes = [vp, c_int, c_int, c_int, vp, vp, c_long]
-    lib.oracle_quantize_blocks.argtypes = [vp, c_int, c_int, c_int, vp, vp]
+    lib.oracle_e5m2_encode_array.argtypes = [vp, c_long, vp]
+    lib.oracle_quantize_rows.argtypes = [vp, c_int, c_int, c_int, vp, vp, c_long, c_int]
+    lib.oracle_quantize_blocks.argtypes = [vp, c_int, c_int, c_int, vp, vp, c_int]
     return lib
 
 
@@ -192,7 +193,15 @@ def e4m3_encode(v) -> np.ndarray:
     return out
 
 
-def quantize_rows(X_bits, ld=None):
+def e5m2_encode(v) -> np.ndarray:
+    """e5m2 codes (uint8) of finite fp32 values: round to nearest, ties to even, saturating."""
+    v = _c(v, np.float32)
+    out = np.empty(v.shape, dtype=np.uint8)
+    _lib().oracle_e5m2_encode_array(_p(v), int(v.size), _p(out))
+    return out
+
+
+def quantize_rows(X_bits, ld=None, fmt="e4m3"):
     """A side of the cast: X_bits bf16 bit patterns [M,K] or [G,M,K] -> (codes of the same shape,
     sfa [KB, ld] or [G, KB, ld]); one fp32 scale per 1x128 block of a row, column-major."""
     X = _c(X_bits, np.uint16)
@@ -204,11 +213,11 @@ def quantize_rows(X_bits, ld=None):
     ld = ld if ld is not None else (M + 3) // 4 * 4
     Q = np.empty(X.shape, dtype=np.uint8)
     sfa = np.zeros((G, KB, ld), dtype=np.float32)
-    _lib().oracle_quantize_rows(_p(X), G, M, K, _p(Q), _p(sfa), ld)
+    _lib().oracle_quantize_rows(_p(X), G, M, K, _p(Q), _p(sfa), ld, _fmt(fmt))
     return (Q[0], sfa[0]) if squeeze else (Q, sfa)
 
 
-def quantize_blocks(X_bits):
+def quantize_blocks(X_bits, fmt="e4m3"):
     """B side of the cast: X_bits bf16 bit patterns [N,K] or [G,N,K] -> (codes, sfb [NB,KB] or
     [G,NB,KB]); one fp32 scale per 128x128 block."""
     X = _c(X_bits, np.uint16)
@@ -218,5 +227,5 @@ def quantize_blocks(X_bits):
     G, N, K = X.shape
     Q = np.empty(X.shape, dtype=np.uint8)
     sfb = np.empty((G, (N + 127) // 128, (K + 127) // 128), dtype=np.float32)
-    _lib().oracle_quantize_blocks(_p(X), G, N, K, _p(Q), _p(sfb))
+    _lib().oracle_quantize_blocks(_p(X), G, N, K, _p(Q), _p(sfb), _fmt(fmt))
     return (Q[0], sfb[0]) if squeeze else (Q, sfb)

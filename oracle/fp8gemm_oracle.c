@@ -279,10 +279,11 @@ void oracle_grouped_masked(const uint8_t *A, const float *sfa, long ld,
  * done separately; news article, senqingzn.com: fine-grained scaling).  The
  * reading taken here, per block (1 x 128 of a row for A, 128 x 128 for B):
  *   amax  = max |x| over the block (fp32; bf16 -> fp32 is exact)
- *   scale = amax / 448 in fp32 (one IEEE round-to-nearest division), or 1 if
- *           amax == 0
- *   code  = e4m3 round-to-nearest-even of the fp32 quotient x / scale,
- *           saturating at +-448 (448 is the largest finite e4m3 value)
+ *   scale = amax / top in fp32 (one IEEE round-to-nearest division), or 1 if
+ *           amax == 0, top = 448 for e4m3 and 57344 for e5m2 (the formats'
+ *           largest finite values)
+ *   code  = round-to-nearest-even of the fp32 quotient x / scale in the target
+ *           format, saturating at +-top
  * ------------------------------------------------------------------------- */
 
 /* e4m3 code of the finite fp32 value v: the nearest of the 127 non-negative
@@ -310,6 +311,34 @@ void oracle_e4m3_encode_array(const float *v, long n, uint8_t *out) {
     for (long i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(v[i]);
 }
 
+/* e5m2 code of the finite fp32 value v: the nearest of the 124 non-negative finite
+ * magnitudes of the e5m2 table (codes 0x00..0x7B, increasing with the code), ties
+ * to the even code, magnitudes above 57344 clamped to 57344. */
+uint8_t oracle_e5m2_encode(float v) {
+    const double *dec = dec_table_fmt(1);
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs((double)v);
+    if (a >= dec[0x7B]) return sign | 0x7B;
+    int lo = 0, hi = 0x7B;                 /* dec[lo] <= a < dec[hi] */
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (dec[mid] <= a) lo = mid; else hi = mid;
+    }
+    const double dl = a - dec[lo], dh = dec[hi] - a;
+    int c;
+    if (dl < dh) c = lo;
+    else if (dh < dl) c = hi;
+    else c = (lo & 1) ? hi : lo;           /* tie: the even code */
+    return sign | (uint8_t)c;
+}
+
+void oracle_e5m2_encode_array(const float *v, long n, uint8_t *out) {
+    for (long i = 0; i < n; ++i) out[i] = oracle_e5m2_encode(v[i]);
+}
+
+/* the cast's target format: fmt 0 e4m3 (largest finite 448), 1 e5m2 (57344) */
+static uint8_t encode_fmt(float v, int fmt) { return fmt == 0 ? oracle_e4m3_encode(v) : oracle_e5m2_encode(v); }
+
 static float bf16_to_f32(uint16_t b) {
     uint32_t u = (uint32_t)b << 16;
     float f;
@@ -317,15 +346,15 @@ static float bf16_to_f32(uint16_t b) {
     return f;
 }
 
-static float block_scale(float amax) {
-    volatile float s = amax / 448.0f;      /* one fp32 division */
+static float block_scale(float amax, int fmt) {
+    volatile float s = fmt == 0 ? amax / 448.0f : amax / 57344.0f;  /* one fp32 division */
     return amax == 0.0f ? 1.0f : s;
 }
 
 /* A side: X is [G][M][K] bf16 (bit patterns), Q the e4m3 codes in the same
  * layout, sfa the scales [G][ceil(K/128)][ld], ld >= M (rows M..ld-1 of each
  * column are not written). */
-void oracle_quantize_rows(const uint16_t *X, int G, int M, int K, uint8_t *Q, float *sfa, long ld) {
+void oracle_quantize_rows(const uint16_t *X, int G, int M, int K, uint8_t *Q, float *sfa, long ld, int fmt) {
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     long rows = (long)G * M;
     #pragma omp parallel for schedule(static)
@@ -340,18 +369,18 @@ void oracle_quantize_rows(const uint16_t *X, int G, int M, int K, uint8_t *Q, fl
                 float a = fabsf(bf16_to_f32(x[k]));
                 if (a > amax) amax = a;
             }
-            const float s = block_scale(amax);
+            const float s = block_scale(amax, fmt);
             sfa[((size_t)g * KB + kb) * ld + m] = s;
             for (int k = k0; k < k1; ++k) {
                 volatile float v = bf16_to_f32(x[k]) / s;   /* one fp32 division */
-                q[k] = oracle_e4m3_encode(v);
+                q[k] = encode_fmt(v, fmt);
             }
         }
     }
 }
 
 /* B side: X is [G][N][K] bf16, Q the codes, sfb the scales [G][ceil(N/128)][ceil(K/128)]. */
-void oracle_quantize_blocks(const uint16_t *X, int G, int N, int K, uint8_t *Q, float *sfb) {
+void oracle_quantize_blocks(const uint16_t *X, int G, int N, int K, uint8_t *Q, float *sfb, int fmt) {
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
     long blocks = (long)G * NB * KB;
@@ -369,12 +398,12 @@ void oracle_quantize_blocks(const uint16_t *X, int G, int N, int K, uint8_t *Q, 
                 float a = fabsf(bf16_to_f32(x[(size_t)n * K + k]));
                 if (a > amax) amax = a;
             }
-        const float s = block_scale(amax);
+        const float s = block_scale(amax, fmt);
         sfb[b] = s;
         for (int n = n0; n < n1; ++n)
             for (int k = k0; k < k1; ++k) {
                 volatile float v = bf16_to_f32(x[(size_t)n * K + k]) / s;
-                q[(size_t)n * K + k] = oracle_e4m3_encode(v);
+                q[(size_t)n * K + k] = encode_fmt(v, fmt);
             }
     }
 }

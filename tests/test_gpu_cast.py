@@ -127,3 +127,39 @@ def test_cast_quotients_exactly_on_e4m3_midpoints(fg, s):
     assert np.all(sfa_ref[0, :nrows] == np.float32(s))
     assert np.array_equal(q.cpu().numpy(), q_ref)
     assert np.array_equal(sfa.cpu().numpy()[:, :nrows], sfa_ref[:, :nrows])
+
+
+@pytest.mark.parametrize("shape", [(7, 272), (33, 1040), (2, 129, 384)])
+def test_cast_e5m2_bit_exact(fg, shape):
+    x = bf16_inputs(shape, 3 * sum(shape))
+    q, s = fg.cast_fp8_rows(x.cuda(), fmt="e5m2")
+    qb, sb = fg.cast_fp8_blocks(x.cuda(), fmt="e5m2")
+    torch.cuda.synchronize()
+    q_ref, s_ref = oracle.quantize_rows(as_bits(x), fmt="e5m2")
+    qb_ref, sb_ref = oracle.quantize_blocks(as_bits(x), fmt="e5m2")
+    M = shape[-2]
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy()[..., :M].view(np.uint32), s_ref[..., :M].view(np.uint32))
+    assert np.array_equal(qb.cpu().numpy(), qb_ref)
+    assert np.array_equal(sb.cpu().numpy().view(np.uint32), sb_ref.view(np.uint32))
+
+
+def test_cast_e5m2_quotients_on_midpoints(fg):
+    d = oracle.e5m2_decode_table()
+    mids = (d[0:0x7B] + d[1:0x7C]) / 2
+    s = 1.5  # amax = 57344 * 1.5 makes the scale exactly 1.5; m * 1.5 is exact in bf16
+    vals = np.concatenate([mids * s, -mids * s]).astype(np.float32)
+    per_row = 127
+    nrows = (len(vals) + per_row - 1) // per_row
+    x = np.zeros((nrows, 128), dtype=np.float32)
+    x[:, 0] = 57344.0 * s
+    flat = np.zeros(nrows * per_row, dtype=np.float32)
+    flat[:len(vals)] = vals
+    x[:, 1:] = flat.reshape(nrows, per_row)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    assert torch.equal(xb.float(), torch.from_numpy(x))
+    q, sfa = fg.cast_fp8_rows(xb.cuda(), fmt="e5m2")
+    torch.cuda.synchronize()
+    q_ref, sfa_ref = oracle.quantize_rows(as_bits(xb), fmt="e5m2")
+    assert np.all(sfa_ref[0, :nrows] == np.float32(s))
+    assert np.array_equal(q.cpu().numpy(), q_ref)

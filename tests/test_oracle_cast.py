@@ -178,3 +178,51 @@ def test_cast_then_gemm_approximates_the_bf16_product():
     # scale semantics: dequantised A = code * scale reproduces x within the e4m3 step
     deq = dec()[A] * np.repeat(sfa[:, :64].T, 128, axis=1)[:, :384]
     assert np.max(np.abs(deq - bf16_bits_to_f32(X))) <= 0.07 * np.abs(bf16_bits_to_f32(X)).max()
+
+
+# ---------------------------------------------------------------------------- e5m2 target
+def dec52():
+    return oracle.e5m2_decode_table()
+
+
+def test_e5m2_encode_round_trips_ties_and_saturation():
+    d = dec52()
+    codes = np.array([c for c in range(256) if ((c >> 2) & 0x1F) != 0x1F], dtype=np.uint8)
+    vals = d[codes].astype(np.float32)
+    vals[codes == 0x80] = -0.0
+    assert np.array_equal(oracle.e5m2_encode(vals), codes)
+    lo = np.arange(0, 0x7B)
+    mid = ((d[lo] + d[lo + 1]) / 2).astype(np.float32)
+    even = np.where(lo % 2 == 0, lo, lo + 1)
+    assert np.array_equal(oracle.e5m2_encode(mid), even.astype(np.uint8))
+    assert np.array_equal(oracle.e5m2_encode(np.nextafter(mid, np.float32(np.inf))), (lo + 1).astype(np.uint8))
+    assert oracle.e5m2_encode(np.array([57344, 60000, 1e30, -1e30], np.float32)).tolist() == [0x7B, 0x7B, 0x7B, 0xFB]
+
+
+def test_e5m2_encode_matches_torch_in_range():
+    rng = np.random.default_rng(23)
+    v = np.concatenate([rng.uniform(-57344, 57344, 200000), rng.standard_normal(200000) * 1e-3,
+                        rng.standard_normal(100000) * 1e-5]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e5m2_encode(v), ref)
+
+
+def test_e5m2_cast_block_max_and_gemm_round_trip():
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((40, 384)).astype(np.float32) * np.float32(1e3)
+    w = rng.standard_normal((136, 384)).astype(np.float32)
+    X, W = f32_to_bf16_bits(x), f32_to_bf16_bits(w)
+    A, sfa = oracle.quantize_rows(X, fmt="e5m2")
+    B, sfb = oracle.quantize_blocks(W, fmt="e5m2")
+    xa = np.abs(bf16_bits_to_f32(X))
+    for kb in range(3):
+        idx = xa[:, kb * 128:(kb + 1) * 128].argmax(axis=1)
+        assert np.all((A[np.arange(40), kb * 128 + idx] & 0x7F) == 0x7B)  # the maximum lands on 57344
+    C = bf16_bits_to_f32(oracle.gemm_nt(A, sfa, B, sfb, fmt_a="e5m2", fmt_b="e5m2")).astype(np.float64)
+    ref = bf16_bits_to_f32(X).astype(np.float64) @ bf16_bits_to_f32(W).astype(np.float64).T
+    assert np.linalg.norm(C - ref) / np.linalg.norm(ref) < 0.1  # two mantissa bits: ~10% per element
+    # with e4m3 the same inputs are closer: the format reaches the codes
+    A4, sfa4 = oracle.quantize_rows(X)
+    B4, sfb4 = oracle.quantize_blocks(W)
+    C4 = bf16_bits_to_f32(oracle.gemm_nt(A4, sfa4, B4, sfb4)).astype(np.float64)
+    assert np.linalg.norm(C4 - ref) < np.linalg.norm(C - ref)

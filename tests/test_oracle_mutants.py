@@ -76,10 +76,12 @@ def test_pins_catch_planted_mistake(name, tmp_path):
 from tests import test_oracle_cast as cast_pins  # noqa: E402
 
 CAST_MUTANTS = {
-    # ties rounded away from zero instead of to even
+    # ties rounded away from zero instead of to even (e4m3, e5m2)
     "cast_ties_away": ("else c = (lo % 2 == 0) ? lo : hi;", "else c = hi;"),
+    "cast_ties_away_e5m2": ("else c = (lo & 1) ? hi : lo;", "else c = hi;"),
     # the inverse scale
-    "cast_inverse_scale": ("volatile float s = amax / 448.0f;", "volatile float s = 448.0f / amax;"),
+    "cast_inverse_scale": ("volatile float s = fmt == 0 ? amax / 448.0f : amax / 57344.0f;",
+                           "volatile float s = fmt == 0 ? 448.0f / amax : 57344.0f / amax;"),
     # non-saturating conversion: magnitudes above 448 become NaN
     "cast_no_saturation": ("if (a >= dec[0x7E]) return sign | 0x7E;",
                            "if (a > dec[0x7E]) return sign | 0x7F; if (a == dec[0x7E]) return sign | 0x7E;"),
@@ -102,6 +104,9 @@ CAST_PINS = [
     cast_pins.test_blocks_agree_with_rows_when_row_maxima_agree,
     cast_pins.test_blocks_max_lands_on_448_per_block,
     cast_pins.test_cast_then_gemm_approximates_the_bf16_product,
+    cast_pins.test_e5m2_encode_round_trips_ties_and_saturation,
+    cast_pins.test_e5m2_encode_matches_torch_in_range,
+    cast_pins.test_e5m2_cast_block_max_and_gemm_round_trip,
 ]
 
 
