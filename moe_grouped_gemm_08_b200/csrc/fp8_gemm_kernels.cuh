@@ -91,6 +91,7 @@ struct SwapParams {
   int n_tiles;     // ceil(N / 128)
   int debug_stall; // test hook: 1 = the MMA thread first waits on a barrier no one arrives at
   uint32_t fmt_bits;  // operand formats in instruction-descriptor position (MMA A = weights)
+  int tile_aligned;   // 1: CTA c takes whole tiles [c*T/P, (c+1)*T/P) (no split tiles, no fix-up)
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -955,8 +956,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int P = gridDim.x;
   const int KB = p.num_kb;
   const int U = p.n_tiles * KB;
-  const int u_begin = sk_begin(blockIdx.x, P, U);
-  const int u_end = sk_begin(blockIdx.x + 1, P, U);
+  // unit range: stream-K (even split of the units, tiles split between CTAs) or, when the host
+  // finds whole tiles cheaper, tile-aligned (an even split of the tiles; no tile is split)
+  const int u_begin = p.tile_aligned
+                          ? static_cast<int>(static_cast<long long>(blockIdx.x) * p.n_tiles / P) * KB
+                          : sk_begin(blockIdx.x, P, U);
+  const int u_end = p.tile_aligned
+                        ? static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.n_tiles / P) * KB
+                        : sk_begin(blockIdx.x + 1, P, U);
 
   const uint64_t pol_w = l2_policy_evict_first();  // each weight byte is read once
   const uint64_t pol_t = l2_policy_evict_last();   // tokens are re-read by every CTA

@@ -353,7 +353,15 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
   if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
   if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
   const long long units = static_cast<long long>(p.n_tiles) * p.num_kb;
-  const int grid = static_cast<int>(units < st->sms ? units : st->sms);
+  int grid = static_cast<int>(units < st->sms ? units : st->sms);
+  // Whole tiles instead of stream-K when that costs at most kSplitOverheadUnits more K blocks on
+  // the busiest CTA than the even split of the units (the split-K publication and fix-up cost
+  // about that much on the decode shapes).
+  constexpr long long kSplitOverheadUnits = 4;
+  const long long aligned_units = (p.n_tiles + st->sms - 1) / st->sms * static_cast<long long>(p.num_kb);
+  const long long split_units = (units + grid - 1) / grid;
+  p.tile_aligned = (p.n_tiles >= st->sms && aligned_units <= split_units + kSplitOverheadUnits) ? 1 : 0;
+  if (p.tile_aligned) grid = st->sms;
   void* args[3] = {&mW, &mT, &p};
   return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(grid), swap_smem_bytes<MP, STAGES>(), stream,
                                                                args, fg::kThreads);
@@ -421,6 +429,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.n_tiles = (N + kBlockM - 1) / kBlockM;
   p.debug_stall = 0;
   p.fmt_bits = 0;  // e4m3 x e4m3
+  p.tile_aligned = 0;
   if (p.n_tiles > kNoAllocCounters) return FG_ERR_UNSUPPORTED;
   // the counters must start at zero; the kernel leaves them at zero, but a call that gave up a
   // wait may not have, so clear the ones this call uses (a memset, no allocation)
