@@ -357,7 +357,10 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
   // Whole tiles instead of stream-K when that costs at most kSplitOverheadUnits more K blocks on
   // the busiest CTA than the even split of the units (the split-K publication and fix-up cost
   // about that much on the decode shapes).
-  constexpr long long kSplitOverheadUnits = 4;
+#ifndef FG_SPLIT_OVERHEAD_UNITS
+#define FG_SPLIT_OVERHEAD_UNITS 8
+#endif
+  constexpr long long kSplitOverheadUnits = FG_SPLIT_OVERHEAD_UNITS;
   const long long aligned_units = (p.n_tiles + st->sms - 1) / st->sms * static_cast<long long>(p.num_kb);
   const long long split_units = (units + grid - 1) / grid;
   p.tile_aligned = (p.n_tiles >= st->sms && aligned_units <= split_units + kSplitOverheadUnits) ? 1 : 0;
