@@ -444,6 +444,8 @@ def run_ours(args, rank, world, local):
     global KERNEL_PATH
     KERNEL_PATH = args.path
     fg.set_dense_path(args.path)
+    if args.tiled_streamk is not None:
+        fg.set_tiled_streamk(args.tiled_streamk)
     name, wl = workload_list(args.workload, args.shape)
     cases = [make_case(w) for w in wl]
     works = [work_of(c) for c in cases]
@@ -608,7 +610,8 @@ def run_ours(args, rank, world, local):
             "config": {"workload": name, "shapes": [w["name"] for w in wl],
                        "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
                        "graph": "each step replayed from a CUDA graph", "parallelism": f"replicas x{world}",
-                       "kernel_path": args.path},
+                       "kernel_path": args.path,
+                       "tiled_streamk": "library default" if args.tiled_streamk is None else args.tiled_streamk},
             "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
             "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
             "roofline": roof,
@@ -640,6 +643,9 @@ def main():
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="kernel selection (fg_set_dense_path): 0 automatic, 1 one-CTA tiled, "
                          "2 swap-AB stream-K, 3 CTA pair")
+    ap.add_argument("--tiled-streamk", type=int, default=None, metavar="BLOCKS",
+                    help="tiled kernel's stream-K tail threshold (fg_set_tiled_streamk): split the last "
+                         "partial wave when it saves more than BLOCKS K blocks; negative: never")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

@@ -39,8 +39,9 @@
  * Ownership: the caller owns every buffer.  The library allocates only in
  * fg_init (a status word, a split-K workspace and its counters), never inside
  * a GEMM call, so calls can be captured into CUDA graphs.  The workspace is
- * per device; GEMM calls that use it must not run concurrently on different
- * streams of the same device.
+ * per device and every GEMM entry point may use it (split tiles of the small-M
+ * kernel and of the tiled kernel's last wave), so GEMM calls must not run
+ * concurrently on different streams of the same device.
  *
  * Errors: every entry point returns a status code and never throws.  Argument
  * errors are found on the host before any launch and launch nothing.  A device
@@ -197,6 +198,18 @@ const char* fg_status_string(fg_status status);
  * always takes the one-CTA tiled kernel.  Returns the previous value; an unknown
  * value is ignored. */
 int fg_set_dense_path(int path);
+
+/* Stream-K tail of the tiled kernel (dense M > 128, contiguous, masked), process-wide.
+ * The tiles are walked whole in waves over the SMs; when the last wave is partial
+ * its tiles are instead split in K over all the CTAs, and a tile split between CTAs
+ * is summed (fp32 partials in the library's workspace, in a fixed CTA order, so the
+ * result does not depend on timing) by the last CTA to finish it.  The split is taken
+ * when the busiest CTA's share of the split units, plus `overhead` K blocks of 128 for
+ * publishing partial tiles (default 18) and 2.4 K blocks per piece summed, is at most
+ * one whole tile; 0 takes it whenever the last wave is partial, a negative value
+ * never.  Returns the previous value.  Results differ from the unsplit walk only in
+ * fp32 summation order. */
+int fg_set_tiled_streamk(int overhead);
 
 /* Failure injection for tests (process-wide, default 0).  With 1, every kernel of
  * fp8_gemm_nt that takes the small-M (swap-AB stream-K) path first waits on a barrier

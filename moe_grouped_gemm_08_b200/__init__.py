@@ -69,6 +69,8 @@ _lib.fg_set_dense_path.argtypes = [_int]
 _lib.fg_set_dense_path.restype = _int
 _lib.fg_debug_set_stall.argtypes = [_int]
 _lib.fg_debug_set_stall.restype = _int
+_lib.fg_set_tiled_streamk.argtypes = [_int]
+_lib.fg_set_tiled_streamk.restype = _int
 _lib.fg_launch_count.argtypes = []
 _lib.fg_launch_count.restype = ctypes.c_uint64
 
@@ -110,6 +112,13 @@ def set_dense_path(path: int) -> int:
     """0 automatic, 1 one-CTA tiled kernel (dense), 2 swap-AB stream-K (dense, M <= 128),
     3 CTA-pair kernel (dense and masked). Returns the old value."""
     return int(_lib.fg_set_dense_path(int(path)))
+
+
+def set_tiled_streamk(overhead: int) -> int:
+    """Stream-K tail of the tiled kernel: split the last partial wave when its cost (its units +
+    `overhead` K blocks + 2.4 per piece summed) is at most one tile (default 18; 0 whenever the last
+    wave is partial; negative never). Returns the old value."""
+    return int(_lib.fg_set_tiled_streamk(int(overhead)))
 
 
 def launch_count() -> int:

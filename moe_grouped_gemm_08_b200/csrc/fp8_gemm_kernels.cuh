@@ -77,6 +77,9 @@ struct TiledParams {
   int n_blocks; // ceil(N / BN)
   int group_m;  // tile order: groups of group_m m-blocks, m-block fastest inside a group
   uint32_t fmt_bits;  // operand formats in instruction-descriptor position (0: both e4m3)
+  float* ws;        // stream-K tail: 2 * gridDim.x partial tiles of 128 x BN fp32
+  int* counters;    // stream-K tail: one per tile of the last partial wave, zero between launches
+  int sk_overhead;  // < 0: no stream-K tail; else the K blocks a split must save to be taken
 };
 
 struct SwapParams {
@@ -124,6 +127,99 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, volat
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Stream-K split of U units (one K block of one tile each, u = t * KB + kb) over P CTAs: CTA c
+// owns units [sk_begin(c), sk_begin(c + 1)); with U >= P every CTA has at least one.  N * K < 2^40
+// keeps the unit count below 2^26, so unit indices fit in 32 bits.
+__device__ __forceinline__ int sk_begin(int c, int P, int U) {
+  return static_cast<int>((static_cast<long long>(c) * U) / P);
+}
+__device__ __forceinline__ int sk_owner(int u, int P, int U) {
+  return static_cast<int>(((static_cast<long long>(u) + 1) * P - 1) / U);
+}
+// Workspace slot of CTA c's piece of the tile whose first unit is tu0.
+// Slot 2c holds the first segment of the CTA's range, slot 2c+1 its last (middle segments are
+// whole tiles and never need a slot).
+__device__ __forceinline__ int sk_slot(int c, int P, int U, int tu0) {
+  return 2 * c + (sk_begin(c, P, U) >= tu0 ? 0 : 1);
+}
+
+// Work of one CTA of the tiled kernel.  Tiles [0, dp_end) are walked whole, CTA c taking tiles
+// c, c + P, ...  When the last partial wave is split (the stream-K tail), its tiles dp_end ..
+// form U = (tiles - dp_end) * KB units, spread over sk_ctas = min(U, P) CTAs so that every one of
+// them has at least one unit; a tile split between CTAs is summed by the last of them to finish.
+// The tail is taken only when its cost on the busiest CTA is at most the whole tile it replaces:
+// its share of the units, plus `overhead` K blocks for publishing partial tiles, plus 2.4 K blocks
+// for each piece the last CTA of a tile sums (the most pieces a tile can have).  overhead = 0
+// takes the tail whenever the last wave is partial.
+__device__ __host__ __forceinline__ bool tiled_tail_pays(int U, int ctas, int KB, int overhead) {
+  const int per = (U + ctas - 1) / ctas;
+  const int pieces = (KB + per - 1) / per + 1;
+  return per + (overhead > 0 ? overhead + (12 * pieces + 4) / 5 : 0) <= KB;
+}
+struct TiledPlan {
+  int dp_end;   // first tile of the stream-K tail (all tiles when there is none)
+  int U;        // units of the tail
+  int sk_ctas;  // CTAs sharing the tail
+  int u_end;    // end of this CTA's unit range
+};
+struct TiledItem {
+  int t;    // tile
+  int kb0;  // K blocks [kb0, kb1) of it
+  int kb1;
+};
+struct TiledCursor {
+  int t;  // next whole tile
+  int u;  // next unit of the tail
+};
+
+__device__ __forceinline__ TiledPlan tiled_plan(int num_tiles, int KB, int overhead, TiledCursor& cur) {
+  const int P = gridDim.x;
+  TiledPlan w;
+  w.dp_end = num_tiles;
+  w.U = 0;
+  w.sk_ctas = 0;
+  w.u_end = 0;
+  cur.t = blockIdx.x;
+  cur.u = 0;
+  const int full = num_tiles / P;
+  const int rem = num_tiles - full * P;
+  if (overhead >= 0 && rem > 0) {
+    const int U = rem * KB;
+    const int ctas = U < P ? U : P;
+    if (tiled_tail_pays(U, ctas, KB, overhead)) {
+      w.dp_end = full * P;
+      w.U = U;
+      w.sk_ctas = ctas;
+      if (static_cast<int>(blockIdx.x) < ctas) {
+        cur.u = sk_begin(blockIdx.x, ctas, U);
+        w.u_end = sk_begin(blockIdx.x + 1, ctas, U);
+      }
+    }
+  }
+  return w;
+}
+
+// Next work item of this CTA (whole tiles first, then its pieces of the tail); false when done.
+__device__ __forceinline__ bool tiled_next(const TiledPlan& w, int KB, TiledCursor& cur, TiledItem& it) {
+  if (cur.t < w.dp_end) {
+    it.t = cur.t;
+    it.kb0 = 0;
+    it.kb1 = KB;
+    cur.t += gridDim.x;
+    return true;
+  }
+  if (cur.u < w.u_end) {
+    const int tl = cur.u / KB;
+    const int e = (w.u_end < (tl + 1) * KB) ? w.u_end : (tl + 1) * KB;
+    it.t = w.dp_end + tl;
+    it.kb0 = cur.u - tl * KB;
+    it.kb1 = e - tl * KB;
+    cur.u = e;
+    return true;
+  }
+  return false;
 }
 
 // ============================================================================
@@ -271,6 +367,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   uint64_t* pbar = mma_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* s_prefix = reinterpret_cast<int*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5;
@@ -328,6 +425,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   } else {
     num_tiles = p.m_blocks * p.n_blocks;
   }
+  TiledCursor cur;
+  const TiledPlan plan = tiled_plan(num_tiles, p.num_kb, p.sk_overhead, cur);
+  TiledItem it;
 
   if (warp >= kPromoWarps) {
     // ================================================ warpgroup 2: producer, MMA, idle warps
@@ -338,12 +438,12 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       bool ok = true;
       const uint64_t pol_a = l2_policy_evict_last();   // A rows: re-read by every n-block of a group
       const uint64_t pol_b = l2_policy_evict_first();  // B tiles: shared by the concurrent m-blocks only
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+      while (ok && tiled_next(plan, p.num_kb, cur, it)) {
+        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, it.t, BN);
         if (!ti.live) continue;
         const int ga = (MODE == kMasked) ? ti.g : 0;
         const int gb = (MODE == kDense) ? 0 : ti.g;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = it.kb0; kb < it.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           uint8_t* st = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
@@ -360,10 +460,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     } else if (warp == kMmaWarp && lane == 0) {
       uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
+      while (ok && tiled_next(plan, p.num_kb, cur, it)) {
+        const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, it.t, BN);
         if (!ti.live) continue;
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = it.kb0; kb < it.kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
@@ -392,40 +492,37 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     const int row = q * 32 + lane;
     const int tid = threadIdx.x;  // 0..255 among promotion threads
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-    const int n_chunks = (p.num_kb + kSaChunk - 1) / kSaChunk;
     uint8_t* s_w = s_out + warp * WARP_STORE_BYTES;  // this warp's output staging
     bool stores_pending = false;
     uint32_t tb = 0, tphase = 0, pphase = 0;
     bool ok = true;
 
-    // first live tile of this CTA
-    int t = blockIdx.x;
+    // next live work item of this CTA
+    auto next_live = [&](TiledItem& item, TileInfo& info) -> bool {
+      while (tiled_next(plan, p.num_kb, cur, item)) {
+        info = tiled_tile<MODE>(p, s_prefix, live_mblocks, item.t, BN);
+        if (info.live) return true;
+      }
+      return false;
+    };
     TileInfo ti;
-    ti.live = 0;
-    for (; t < num_tiles; t += gridDim.x) {
-      ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, t, BN);
-      if (ti.live) break;
-    }
-    // Scale chunks form one sequence over this CTA's tiles; chunk X lives in s_scale[X % 2].
-    // The registers hold the chunk after the one being processed; it is stored into the other
-    // slot once this chunk is done, which is safe because the barrier that ended the previous
-    // chunk guarantees that no thread still reads that slot.
+    bool have = next_live(it, ti);
+    // Scale chunks (kSaChunk K blocks each) form one sequence over this CTA's work items; chunk X
+    // of the sequence lives in s_scale[X % 2].  The registers hold the chunk after the one being
+    // processed; it is stored into the other slot once this chunk is done, which is safe because
+    // the barrier that ended the previous chunk guarantees that no thread still reads that slot.
     ScaleChunkRegs nxt;
     int buf = 0;
-    if (t < num_tiles) {
-      load_scale_chunk<MODE>(p, ti, 0, tid, nxt);
+    if (have) {
+      load_scale_chunk<MODE>(p, ti, it.kb0 / kSaChunk, tid, nxt);
       store_scale_chunk(s_scale, tid, nxt);
       ok = group_sync(pbar, pphase, abort_flag);
     }
-    while (t < num_tiles && ok) {
-      // the tile after this one (for the chunk prefetch that crosses tiles)
-      int t_next = t + gridDim.x;
+    while (have && ok) {
+      // the item after this one (for the chunk prefetch that crosses items)
+      TiledItem it_next;
       TileInfo ti_next;
-      ti_next.live = 0;
-      for (; t_next < num_tiles; t_next += gridDim.x) {
-        ti_next = tiled_tile<MODE>(p, s_prefix, live_mblocks, t_next, BN);
-        if (ti_next.live) break;
-      }
+      const bool have_next = next_live(it_next, ti_next);
       const int m = ti.m0 + row;
       // sfb block (0: the tile's first, 1: the next) of each 32-column chunk of this thread
       uint32_t hi_mask = 0;
@@ -437,14 +534,17 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 #pragma unroll
       for (int j = 0; j < COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
 
-      for (int c = 0; c < n_chunks && ok; ++c) {
+      const int c_lo = it.kb0 / kSaChunk;
+      const int c_hi = (it.kb1 - 1) / kSaChunk;
+      for (int c = c_lo; c <= c_hi && ok; ++c) {
         // prefetch the next chunk of the sequence into registers
-        if (c + 1 < n_chunks) load_scale_chunk<MODE>(p, ti, c + 1, tid, nxt);
-        else if (t_next < num_tiles) load_scale_chunk<MODE>(p, ti_next, 0, tid, nxt);
+        if (c < c_hi) load_scale_chunk<MODE>(p, ti, c + 1, tid, nxt);
+        else if (have_next) load_scale_chunk<MODE>(p, ti_next, it_next.kb0 / kSaChunk, tid, nxt);
         const float* sa = s_scale + buf * CHUNK_FLOATS + row;
         const float* sb = s_scale + buf * CHUNK_FLOATS + kSaChunk * kBlockM;
-        const int kb_end = (c + 1) * kSaChunk < p.num_kb ? (c + 1) * kSaChunk : p.num_kb;
-        for (int kb = c * kSaChunk; kb < kb_end; ++kb) {
+        const int kb_begin = c * kSaChunk > it.kb0 ? c * kSaChunk : it.kb0;
+        const int kb_end = (c + 1) * kSaChunk < it.kb1 ? (c + 1) * kSaChunk : it.kb1;
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           const int kl = kb - c * kSaChunk;
           const float sav = sa[kl * kBlockM];
           const float s0 = sav * sb[kl];
@@ -474,11 +574,59 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         if (!ok) break;
         // publish the prefetched chunk into the other slot, then one barrier
         const int nbuf = buf ^ 1;
-        if (c + 1 < n_chunks || t_next < num_tiles) store_scale_chunk(s_scale + nbuf * CHUNK_FLOATS, tid, nxt);
+        if (c < c_hi || have_next) store_scale_chunk(s_scale + nbuf * CHUNK_FLOATS, tid, nxt);
         if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
         buf = nbuf;
       }
       if (!ok) break;
+
+      if (it.kb0 != 0 || it.kb1 != p.num_kb) {
+        // A piece of a split tile of the stream-K tail: publish the fp32 partial; the last CTA of
+        // the tile to arrive sums every piece in CTA order (so results are bit-reproducible) and
+        // writes the tile.  No CTA ever waits for another.  Thread tid's values sit at float4
+        // positions i * 256 + tid of a partial, the same in every CTA.
+        constexpr int TILE_F4 = kBlockM * BN / 4;
+        const int tl = it.t - plan.dp_end;
+        const int tu0 = tl * p.num_kb;
+        const int c_first = sk_owner(tu0, plan.sk_ctas, plan.U);
+        const int c_last = sk_owner(tu0 + p.num_kb - 1, plan.sk_ctas, plan.U);
+        float4* ws4 = reinterpret_cast<float4*>(p.ws);
+        float4* wp = ws4 + static_cast<size_t>(sk_slot(blockIdx.x, plan.sk_ctas, plan.U, tu0)) * TILE_F4 + tid;
+#pragma unroll
+        for (int i = 0; i < COLS / 4; ++i)
+          wp[i * kPromoWarps * 32] = make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x, acc[2 * i + 1].y);
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        if (tid == 0) {
+          fence_acq_rel_gpu();  // release this CTA's partial (ordered before by the barrier)
+          const int prev = atomicAdd(p.counters + tl, 1);
+          const int last = (prev == c_last - c_first);
+          if (last) {
+            fence_acq_rel_gpu();  // acquire the other CTAs' partials
+            p.counters[tl] = 0;   // ready for the next launch
+          }
+          *s_last = last;
+        }
+        if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+        if (!*s_last) {
+          it = it_next;
+          ti = ti_next;
+          have = have_next;
+          continue;
+        }
+#pragma unroll
+        for (int j = 0; j < COLS / 2; ++j) acc[j] = make_float2(0.0f, 0.0f);
+        for (int c = c_first; c <= c_last; ++c) {
+          const float4* src = ws4 + static_cast<size_t>(sk_slot(c, plan.sk_ctas, plan.U, tu0)) * TILE_F4 + tid;
+#pragma unroll
+          for (int i = 0; i < COLS / 4; ++i) {
+            const float4 a = __ldcg(src + i * kPromoWarps * 32);
+            acc[2 * i].x += a.x;
+            acc[2 * i].y += a.y;
+            acc[2 * i + 1].x += a.z;
+            acc[2 * i + 1].y += a.w;
+          }
+        }
+      }
 
       // epilogue: bf16 round-to-nearest-even.  A warp whose 32 rows are all to be written stages
       // them in shared memory and stores them with TMA; a warp with rows that must stay untouched
@@ -543,8 +691,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           }
         }
       }
-      t = t_next;
+      it = it_next;
       ti = ti_next;
+      have = have_next;
     }
     if (stores_pending && lane == 0) bulk_wait_all();
   }
@@ -903,21 +1052,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
 // ============================================================================
 // Kernel 2: swap-AB stream-K (dense, M <= MP <= 128)
 // ============================================================================
-// Units are (n-tile, K block) pairs, u = t * KB + kb; CTA c owns units [begin(c), begin(c+1)).
-// N * K < 2^40 keeps the unit count below 2^26, so unit indices fit in 32 bits.
-__device__ __forceinline__ int sk_begin(int c, int P, int U) {
-  return static_cast<int>((static_cast<long long>(c) * U) / P);
-}
-__device__ __forceinline__ int sk_owner(int u, int P, int U) {
-  return static_cast<int>(((static_cast<long long>(u) + 1) * P - 1) / U);
-}
-// Workspace slot of CTA c's piece of the tile whose first unit is tu0.
-// Slot 2c holds the first segment of the CTA's range, slot 2c+1 its last (middle segments are
-// whole tiles and never need a slot).
-__device__ __forceinline__ int sk_slot(int c, int P, int U, int tu0) {
-  return 2 * c + (sk_begin(c, P, U) >= tu0 ? 0 : 1);
-}
-
+// Units are (n-tile, K block) pairs split over the CTAs with sk_begin.
 template <int MP, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_swap_streamk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,

@@ -40,6 +40,14 @@ DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
 std::atomic<int> g_dense_path{0};
 std::atomic<int> g_debug_stall{0};
+// Tiled kernel: the last partial wave of tiles is split in K over all CTAs (stream-K tail) when
+// its cost on the busiest CTA -- its units, this many K blocks for publishing partial tiles (a
+// CTA may publish twice, about 3.4 us = 7 K blocks each, measured) and 2.4 K blocks per piece
+// summed -- is at most the tile it replaces; 0: whenever the last wave is partial; negative: never.
+#ifndef FG_TILED_SK_OVERHEAD
+#define FG_TILED_SK_OVERHEAD 18
+#endif
+std::atomic<int> g_tiled_sk{FG_TILED_SK_OVERHEAD};
 std::atomic<uint64_t> g_launches{0};
 
 // tiled kernel configuration: 128 x 192 output tiles, 4-stage ring (overridable when building)
@@ -243,8 +251,20 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
   if (!encode_fp8_map(&mB, B, K, N, groupsB, BN)) return FG_ERR_CUDA;
   if (!encode_bf16_store_map(&mC, C, N, M, groupsA, MODE == fg::kMasked)) return FG_ERR_CUDA;
 
-  long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
-  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  p.ws = st->ws;
+  p.counters = st->counters;
+  p.sk_overhead = g_tiled_sk.load(std::memory_order_relaxed);
+  // masked: an upper bound (the live tiles are counted on the device)
+  const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
+  int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  if (tiles < st->sms && p.sk_overhead >= 0) {
+    // fewer tiles than SMs: the kernel splits them in K over more CTAs if that pays (the same
+    // test the kernel makes)
+    const long long units = tiles * p.num_kb;
+    const long long ctas = units < st->sms ? units : st->sms;
+    if (fg::tiled_tail_pays(static_cast<int>(units), static_cast<int>(ctas), p.num_kb, p.sk_overhead))
+      grid = static_cast<int>(ctas);
+  }
   void* args[4] = {&mA, &mB, &mC, &p};
   return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, MODE>>(dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, args,
                                                               fg::kTiledThreads, fg::kTiledLaunchRegs);
@@ -288,6 +308,9 @@ fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void*
   constexpr size_t SMEM = pair_smem_bytes<BN, STAGES>();
   fg::TiledParams p;
   p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
+  p.ws = nullptr;
+  p.counters = nullptr;
+  p.sk_overhead = -1;
   p.sfa = sfa;
   p.sfb = sfb;
   p.C = static_cast<__nv_bfloat16*>(C);
@@ -476,7 +499,9 @@ fg_status fg_init(int device) {
     return FG_ERR_CUDA;
   if (major != 10 || minor != 0) return FG_ERR_UNSUPPORTED;  // built for sm_100a only
   if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return FG_ERR_CUDA;
-  const size_t ws_floats = static_cast<size_t>(2) * st.sms * kMaxSwapMP * kBlockM;
+  // two partial tiles per CTA: MP x 128 (swap kernel) or 128 x BN (tiled kernel's stream-K tail)
+  const size_t tile_floats = static_cast<size_t>(kBlockM) * (kMaxSwapMP > kTiledBN ? kMaxSwapMP : kTiledBN);
+  const size_t ws_floats = static_cast<size_t>(2) * st.sms * tile_floats;
   if (cudaMalloc(&st.status, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
   if (cudaMalloc(&st.ws, ws_floats * sizeof(float)) != cudaSuccess) return FG_ERR_CUDA;
   if (cudaMalloc(&st.counters, kCounterCapacity * sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
@@ -515,6 +540,8 @@ int fg_set_dense_path(int path) {
 uint64_t fg_launch_count(void) { return g_launches.load(); }
 
 int fg_debug_set_stall(int enable) { return g_debug_stall.exchange(enable ? 1 : 0); }
+
+int fg_set_tiled_streamk(int overhead) { return g_tiled_sk.exchange(overhead < 0 ? -1 : overhead); }
 
 static bool valid_formats(int fmt_a, int fmt_b) {
   return (fmt_a == FG_E4M3 || fmt_a == FG_E5M2) && (fmt_b == FG_E4M3 || fmt_b == FG_E5M2);
