@@ -446,6 +446,8 @@ def run_ours(args, rank, world, local):
     fg.set_dense_path(args.path)
     if args.tiled_streamk is not None:
         fg.set_tiled_streamk(args.tiled_streamk)
+    if args.swap_schedule is not None:
+        fg.set_swap_schedule(args.swap_schedule)
     name, wl = workload_list(args.workload, args.shape)
     cases = [make_case(w) for w in wl]
     works = [work_of(c) for c in cases]
@@ -536,6 +538,9 @@ def run_ours(args, rank, world, local):
                        "pages_gbs": round(wk[2] / (ms * 1e-3) / 1e9, 1),
                        "bound": "hbm" if wk[1] / (peaks["hbm_gbs"] * 1e9) > wk[0] / (fp8_peak * 1e12) else "tensor",
                        "roofline_frac": round(t_roof / (ms * 1e-3), 3), "kernel": kernel_name(c)})
+        if kernel_name(c) == "fp8_gemm_swap_streamk_kernel":
+            plan = fg.swap_plan(c["M"], c["N"], c["K"])
+            shapes[-1]["schedule"] = {0: "stream-K", 1: "whole tiles"}.get(plan, f"cluster x{plan}")
         sum_ms_all += ms
         if kernel_name(c) == kernel_name(cases[0]):
             sum_bytes_swap += wk[1]
@@ -611,7 +616,8 @@ def run_ours(args, rank, world, local):
                        "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
                        "graph": "each step replayed from a CUDA graph", "parallelism": f"replicas x{world}",
                        "kernel_path": args.path,
-                       "tiled_streamk": "library default" if args.tiled_streamk is None else args.tiled_streamk},
+                       "tiled_streamk": "library default" if args.tiled_streamk is None else args.tiled_streamk,
+                       "swap_schedule": "library default" if args.swap_schedule is None else args.swap_schedule},
             "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
             "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
             "roofline": roof,
@@ -646,6 +652,9 @@ def main():
     ap.add_argument("--tiled-streamk", type=int, default=None, metavar="BLOCKS",
                     help="tiled kernel's stream-K tail threshold (fg_set_tiled_streamk): split the last "
                          "partial wave when it saves more than BLOCKS K blocks; negative: never")
+    ap.add_argument("--swap-schedule", type=int, default=None, choices=[-1, 0, 2, 4, 8],
+                    help="small-M kernel schedule (fg_set_swap_schedule): 0 automatic, -1 never the "
+                         "cluster split, 2/4/8 the cluster split with that many CTAs per tile")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

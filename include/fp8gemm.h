@@ -211,6 +211,23 @@ int fg_set_dense_path(int path);
  * fp32 summation order. */
 int fg_set_tiled_streamk(int overhead);
 
+/* Schedule of the small-M (swap-AB) kernel, process-wide.  0 (default): automatic --
+ * whole 128-row weight tiles per CTA, stream-K (K blocks split evenly over the CTAs,
+ * split tiles summed through global memory by the last CTA to finish), or a cluster
+ * split: a thread-block cluster of S CTAs per weight tile, each CTA taking 1/S of the
+ * K blocks, the partials summed through distributed shared memory (possible when every
+ * tile's cluster can be resident at once and K has at least S blocks of 128); the
+ * cheapest by a cost model in K blocks.  -1: never the cluster split.  2, 4 or 8: the
+ * cluster split with that S wherever it is possible.  Other values are ignored.  All
+ * schedules sum in a fixed order.  Returns the previous value. */
+int fg_set_swap_schedule(int schedule);
+
+/* The schedule the small-M kernel takes for a dense call of this shape on the current
+ * device under the current setting: S (2, 4 or 8) for the cluster split, 1 for whole
+ * tiles per CTA, 0 for stream-K; -1 if M is not in 1..128, N or K is not positive, or
+ * fg_init has not been called for the device.  Launches nothing. */
+int fg_swap_plan(int M, int N, int K);
+
 /* Failure injection for tests (process-wide, default 0).  With 1, every kernel of
  * fp8_gemm_nt that takes the small-M (swap-AB stream-K) path first waits on a barrier
  * that no one arrives at; the bounded wait runs out after about two seconds, the

@@ -71,6 +71,10 @@ _lib.fg_debug_set_stall.argtypes = [_int]
 _lib.fg_debug_set_stall.restype = _int
 _lib.fg_set_tiled_streamk.argtypes = [_int]
 _lib.fg_set_tiled_streamk.restype = _int
+_lib.fg_set_swap_schedule.argtypes = [_int]
+_lib.fg_set_swap_schedule.restype = _int
+_lib.fg_swap_plan.argtypes = [_int, _int, _int]
+_lib.fg_swap_plan.restype = _int
 _lib.fg_launch_count.argtypes = []
 _lib.fg_launch_count.restype = ctypes.c_uint64
 
@@ -119,6 +123,18 @@ def set_tiled_streamk(overhead: int) -> int:
     `overhead` K blocks + 2.4 per piece summed) is at most one tile (default 18; 0 whenever the last
     wave is partial; negative never). Returns the old value."""
     return int(_lib.fg_set_tiled_streamk(int(overhead)))
+
+
+def set_swap_schedule(schedule: int) -> int:
+    """Small-M kernel schedule: 0 automatic, -1 never the cluster split, 2/4/8 the cluster split
+    with that many CTAs per weight tile wherever possible. Returns the old value."""
+    return int(_lib.fg_set_swap_schedule(int(schedule)))
+
+
+def swap_plan(M: int, N: int, K: int) -> int:
+    """Schedule of the small-M kernel for this dense shape: S (2/4/8) cluster split, 1 whole tiles,
+    0 stream-K, -1 not applicable."""
+    return int(_lib.fg_swap_plan(int(M), int(N), int(K)))
 
 
 def launch_count() -> int:

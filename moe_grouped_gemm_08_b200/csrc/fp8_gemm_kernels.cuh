@@ -95,6 +95,8 @@ struct SwapParams {
   int debug_stall; // test hook: 1 = the MMA thread first waits on a barrier no one arrives at
   uint32_t fmt_bits;  // operand formats in instruction-descriptor position (MMA A = weights)
   int tile_aligned;   // 1: CTA c takes whole tiles [c*T/P, (c+1)*T/P) (no split tiles, no fix-up)
+  int cluster;        // S > 1: the S CTAs of cluster t split tile t in K and sum it through
+                      // distributed shared memory (launched with cluster dims S, grid = tiles * S)
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -1052,7 +1054,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
 // ============================================================================
 // Kernel 2: swap-AB stream-K (dense, M <= MP <= 128)
 // ============================================================================
-// Units are (n-tile, K block) pairs split over the CTAs with sk_begin.
+// Units are (n-tile, K block) pairs split over the CTAs with sk_begin, or whole tiles per CTA
+// (tile_aligned), or -- with cluster = S > 1 -- one tile per cluster of S CTAs, CTA r of the
+// cluster taking K blocks [r KB / S, (r+1) KB / S): each CTA leaves its fp32 partial tile in its
+// own shared memory, and after a cluster barrier CTA r sums rows [r 128/S, (r+1) 128/S) of the
+// tile over the S partials (in rank order, so results are bit-reproducible) through distributed
+// shared memory and writes them; a second cluster barrier keeps every CTA's shared memory alive
+// until its peers have read it.  Every thread reaches both barriers, also after an abort.
 template <int MP, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_swap_streamk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
@@ -1093,10 +1101,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int U = p.n_tiles * KB;
   // unit range: stream-K (even split of the units, tiles split between CTAs) or, when the host
   // finds whole tiles cheaper, tile-aligned (an even split of the tiles; no tile is split)
-  const int u_begin = p.tile_aligned
+  const int S = p.cluster;
+  const int cl_tile = static_cast<int>(blockIdx.x) / S;
+  const int cl_rank = static_cast<int>(blockIdx.x) - cl_tile * S;  // = %cluster_ctarank for cluster dims (S,1,1)
+  const int u_begin = S > 1 ? cl_tile * KB + cl_rank * KB / S
+                      : p.tile_aligned
                           ? static_cast<int>(static_cast<long long>(blockIdx.x) * p.n_tiles / P) * KB
                           : sk_begin(blockIdx.x, P, U);
-  const int u_end = p.tile_aligned
+  const int u_end = S > 1 ? cl_tile * KB + (cl_rank + 1) * KB / S
+                    : p.tile_aligned
                         ? static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.n_tiles / P) * KB
                         : sk_begin(blockIdx.x + 1, P, U);
 
@@ -1277,6 +1290,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_base = t * kBlockM;
       if (kb0 == 0 && kb1 == KB) {  // whole tile
         if (!store_tile(acc, n_base)) { ok = false; break; }
+      } else if (S > 1) {
+        // the cluster's piece of its tile: the fp32 partial goes into this CTA's idle ring
+        // ([token][weight row]; every load has landed and every MMA that read the ring is done)
+        fence_proxy_async_smem();
+        float* part = reinterpret_cast<float*>(smem);
+#pragma unroll
+        for (int j = 0; j < COLS; ++j) part[(h * COLS + j) * kBlockM + nl] = acc[j];
       } else {
         // split tile: the CTAs of the tile publish their fp32 partials; the last to arrive
         // (counter per tile) sums them in CTA order -- so results are bit-reproducible -- and
@@ -1380,6 +1400,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       first_segment = false;
       u = tu0 + kb1;
     }
+  }
+
+  if (S > 1) {
+    // cluster split-K: sum rows [cl_rank R, (cl_rank + 1) R) of the tile over the S partials
+    __syncwarp();
+    cluster_sync_all();  // every CTA's partial is in its shared memory
+    if (warp < kPromoWarps && !*abort_flag) {
+      const int tid = threadIdx.x;
+      const int R4 = kBlockM / S / 4;  // float4 per token row of this CTA's slice
+      const int n_base = cl_tile * kBlockM;
+      const int rows = p.M < MP ? p.M : MP;
+      const uint32_t part = smem_addr(smem);
+      for (int f = tid; f < rows * R4; f += NPROMO) {
+        const int mm = f / R4;
+        const int col = cl_rank * (kBlockM / S) + (f - mm * R4) * 4;
+        if (n_base + col < p.N) {  // N % 8 == 0, so the 4 columns are all inside
+          const uint32_t off = part + static_cast<uint32_t>((mm * kBlockM + col) * 4);
+          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int q = 0; q < S; ++q) {
+            const float4 v = ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)));
+            r.x += v.x; r.y += v.y; r.z += v.z; r.w += v.w;
+          }
+          uint2 val;
+          val.x = pack_bf16x2(r.x, r.y);
+          val.y = pack_bf16x2(r.z, r.w);
+          *reinterpret_cast<uint2*>(p.C + static_cast<size_t>(mm) * p.N + n_base + col) = val;
+        }
+      }
+    }
+    __syncwarp();
+    cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
   }
 
   tc_fence_before();

@@ -48,6 +48,9 @@ std::atomic<int> g_debug_stall{0};
 #define FG_TILED_SK_OVERHEAD 18
 #endif
 std::atomic<int> g_tiled_sk{FG_TILED_SK_OVERHEAD};
+// Small-M kernel schedule: 0 automatic, -1 never a cluster split, 2/4/8 the cluster split with
+// that many CTAs per tile wherever it is possible.
+std::atomic<int> g_swap_schedule{0};
 std::atomic<uint64_t> g_launches{0};
 
 // tiled kernel configuration: 128 x 192 output tiles, 4-stage ring (overridable when building)
@@ -161,7 +164,8 @@ bool encode_fp8_map_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t 
 // build where the compiler chose another count (the split would never be granted).
 // args: pointers to the kernel's arguments, in order.
 template <auto KERNEL>
-fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, void** args, int threads, int required_regs = 0) {
+fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, void** args, int threads, int required_regs = 0,
+                 int cluster = 1) {
   // the opt-in shared-memory size is a per-function attribute: set once per device (so that a
   // call made during stream capture issues no attribute change)
   const auto kernel = KERNEL;
@@ -182,9 +186,14 @@ fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, void** args, int t
   // programmatic dependent launch: the kernel's prologue (barriers, TMEM allocation, descriptor
   // prefetch) may overlap the previous kernel of the stream; the kernel waits for that kernel
   // (griddepcontrol.wait) before its first global-memory access
-  cudaLaunchAttribute attr[1];
+  // cluster > 1: thread-block clusters of that many CTAs along x (grid.x is a multiple of it)
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = grid;
@@ -192,7 +201,7 @@ fg_status launch(dim3 grid, size_t smem, cudaStream_t stream, void** args, int t
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = cluster > 1 ? 2 : 1;
   cudaError_t e = cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(kernel), args);
   if (e != cudaSuccess) return FG_ERR_CUDA;
   g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -350,6 +359,100 @@ fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void*
                         fg::kTiledLaunchRegs);
 }
 
+// Largest number of clusters of `size` CTAs of KERNEL that can be resident at once (clusters must
+// fit inside a GPC, so this can be below #SMs / size); queried once per device, kernel and size.
+template <auto KERNEL>
+int cluster_capacity(int size, int threads, size_t smem) {
+  static std::atomic<int> cached[kMaxDevices][4];
+  const int dev = current_device();
+  const int slot = size == 2 ? 0 : size == 4 ? 1 : size == 8 ? 2 : 3;
+  if (dev < 0 || dev >= kMaxDevices || slot == 3) return 0;
+  int v = cached[dev][slot].load(std::memory_order_acquire);
+  if (v != 0) return v < 0 ? 0 : v;
+  // the query needs the kernel's opt-in shared-memory size in place
+  if (cudaFuncSetAttribute(KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(size);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(static_cast<unsigned>(size), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, KERNEL, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached[dev][slot].store(n > 0 ? n : -1, std::memory_order_release);
+  return n;
+}
+
+struct SwapChoice {
+  int grid;
+  int tile_aligned;
+  int cluster;
+};
+
+// Schedule of the small-M kernel for n_tiles weight tiles of 128 rows and num_kb K blocks.
+// Whole tiles instead of stream-K when that costs at most kSplitOverheadUnits more K blocks on the
+// busiest CTA than the even split of the units (the split-K publication and fix-up cost about
+// that much on the decode shapes).  Cluster split-K: S CTAs per tile, all tiles resident at once
+// (tiles <= the cluster capacity), each CTA with at least one K block.  Cost model in K blocks on
+// the busiest CTA: the cluster split pays ceil(KB / S) + FG_SWAP_CLUSTER_UNITS; stream-K its share
+// + FG_SWAP_STREAMK_UNITS (publishing a partial through global memory and the last CTA's sum of
+// the pieces); tile-aligned ranges their whole tiles.
+#ifndef FG_SPLIT_OVERHEAD_UNITS
+#define FG_SPLIT_OVERHEAD_UNITS 8
+#endif
+#ifndef FG_SWAP_CLUSTER_UNITS
+#define FG_SWAP_CLUSTER_UNITS 2
+#endif
+#ifndef FG_SWAP_STREAMK_UNITS
+#define FG_SWAP_STREAMK_UNITS 16
+#endif
+template <int MP>
+SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
+  constexpr int STAGES = swap_stages<MP>();
+  constexpr auto KERNEL = fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>;
+  constexpr size_t SMEM = swap_smem_bytes<MP, STAGES>();
+  constexpr long long kSplitOverheadUnits = FG_SPLIT_OVERHEAD_UNITS;
+  SwapChoice c;
+  const long long units = static_cast<long long>(n_tiles) * num_kb;
+  c.grid = static_cast<int>(units < sms ? units : sms);
+  const long long aligned_units = (n_tiles + sms - 1) / sms * static_cast<long long>(num_kb);
+  const long long split_units = (units + c.grid - 1) / c.grid;
+  c.tile_aligned = (n_tiles >= sms && aligned_units <= split_units + kSplitOverheadUnits) ? 1 : 0;
+  if (c.tile_aligned) c.grid = sms;
+  c.cluster = 1;
+  const int sched = g_swap_schedule.load(std::memory_order_relaxed);
+  if (sched >= 0) {
+    long long best = c.tile_aligned ? aligned_units : (split_units + (num_kb > 1 ? FG_SWAP_STREAMK_UNITS : 0));
+    for (int S : {8, 4, 2}) {
+      if (sched > 0 && S != sched) continue;
+      if (S > num_kb || n_tiles > cluster_capacity<KERNEL>(S, fg::kThreads, SMEM)) continue;
+      const long long cost = (num_kb + S - 1) / S + FG_SWAP_CLUSTER_UNITS;
+      if (sched > 0 || cost < best) {
+        best = cost;
+        c.cluster = S;
+      }
+    }
+  }
+  if (c.cluster > 1) {
+    c.tile_aligned = 0;
+    c.grid = n_tiles * c.cluster;
+  }
+  return c;
+}
+
 template <int MP>
 fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
@@ -375,22 +478,12 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
   CUtensorMap mW, mT;
   if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
   if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
-  const long long units = static_cast<long long>(p.n_tiles) * p.num_kb;
-  int grid = static_cast<int>(units < st->sms ? units : st->sms);
-  // Whole tiles instead of stream-K when that costs at most kSplitOverheadUnits more K blocks on
-  // the busiest CTA than the even split of the units (the split-K publication and fix-up cost
-  // about that much on the decode shapes).
-#ifndef FG_SPLIT_OVERHEAD_UNITS
-#define FG_SPLIT_OVERHEAD_UNITS 8
-#endif
-  constexpr long long kSplitOverheadUnits = FG_SPLIT_OVERHEAD_UNITS;
-  const long long aligned_units = (p.n_tiles + st->sms - 1) / st->sms * static_cast<long long>(p.num_kb);
-  const long long split_units = (units + grid - 1) / grid;
-  p.tile_aligned = (p.n_tiles >= st->sms && aligned_units <= split_units + kSplitOverheadUnits) ? 1 : 0;
-  if (p.tile_aligned) grid = st->sms;
+  const SwapChoice c = swap_choose<MP>(st->sms, p.n_tiles, p.num_kb);
+  p.tile_aligned = c.tile_aligned;
+  p.cluster = c.cluster;
   void* args[3] = {&mW, &mT, &p};
-  return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(grid), swap_smem_bytes<MP, STAGES>(), stream,
-                                                               args, fg::kThreads);
+  return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(c.grid), swap_smem_bytes<MP, STAGES>(), stream,
+                                                               args, fg::kThreads, 0, c.cluster);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -456,6 +549,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.debug_stall = 0;
   p.fmt_bits = 0;  // e4m3 x e4m3
   p.tile_aligned = 0;
+  p.cluster = 1;
   if (p.n_tiles > kNoAllocCounters) return FG_ERR_UNSUPPORTED;
   // the counters must start at zero; the kernel leaves them at zero, but a call that gave up a
   // wait may not have, so clear the ones this call uses (a memset, no allocation)
@@ -542,6 +636,24 @@ uint64_t fg_launch_count(void) { return g_launches.load(); }
 int fg_debug_set_stall(int enable) { return g_debug_stall.exchange(enable ? 1 : 0); }
 
 int fg_set_tiled_streamk(int overhead) { return g_tiled_sk.exchange(overhead < 0 ? -1 : overhead); }
+
+int fg_swap_plan(int M, int N, int K) {
+  if (M <= 0 || M > kMaxSwapMP || N <= 0 || K <= 0) return -1;
+  fg_status err;
+  DeviceState* st = state_for_current(&err);
+  if (!st) return -1;
+  const int tiles = (N + kBlockM - 1) / kBlockM;
+  const int kb = (K + kBlockK - 1) / kBlockK;
+  const SwapChoice c = M <= 32 ? swap_choose<32>(st->sms, tiles, kb)
+                       : M <= 64 ? swap_choose<64>(st->sms, tiles, kb) : swap_choose<128>(st->sms, tiles, kb);
+  return c.cluster > 1 ? c.cluster : c.tile_aligned;
+}
+
+int fg_set_swap_schedule(int schedule) {
+  if (schedule != 0 && schedule != -1 && schedule != 2 && schedule != 4 && schedule != 8)
+    return g_swap_schedule.load();
+  return g_swap_schedule.exchange(schedule);
+}
 
 static bool valid_formats(int fmt_a, int fmt_b) {
   return (fmt_a == FG_E4M3 || fmt_a == FG_E5M2) && (fmt_b == FG_E4M3 || fmt_b == FG_E5M2);
