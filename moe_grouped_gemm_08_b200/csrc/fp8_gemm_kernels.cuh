@@ -1061,6 +1061,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
 // tile over the S partials (in rank order, so results are bit-reproducible) through distributed
 // shared memory and writes them; a second cluster barrier keeps every CTA's shared memory alive
 // until its peers have read it.  Every thread reaches both barriers, also after an abort.
+// Cluster split-K reduction of the swap kernel: this CTA (rank `rank` of S) sums weight rows
+// [rank 128/S, (rank+1) 128/S) of the tile over the S partials ([token][weight row] fp32 at shared
+// address `part` in every CTA of the cluster), in rank order, and stores them as bf16.  All S
+// loads of an element are issued before the sum.
+template <int S, int MP>
+__device__ __forceinline__ void cluster_reduce_store(const SwapParams& p, uint32_t part, int rank, int n_base,
+                                                     int tid) {
+  constexpr int R4 = kBlockM / S / 4;  // float4 per token row of this CTA's slice
+  constexpr int NPROMO = kPromoWarps * 32;
+  const int rows = p.M < MP ? p.M : MP;
+#pragma unroll 2
+  for (int f = tid; f < rows * R4; f += NPROMO) {
+    const int mm = f / R4;
+    const int col = rank * (kBlockM / S) + (f - mm * R4) * 4;
+    const uint32_t off = part + static_cast<uint32_t>((mm * kBlockM + col) * 4);
+    float4 v[S];
+#pragma unroll
+    for (int q = 0; q < S; ++q) v[q] = ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)));
+    float4 r = v[0];
+#pragma unroll
+    for (int q = 1; q < S; ++q) {
+      r.x += v[q].x; r.y += v[q].y; r.z += v[q].z; r.w += v[q].w;
+    }
+    if (n_base + col < p.N) {  // N % 8 == 0, so the 4 columns are all inside
+      uint2 val;
+      val.x = pack_bf16x2(r.x, r.y);
+      val.y = pack_bf16x2(r.z, r.w);
+      *reinterpret_cast<uint2*>(p.C + static_cast<size_t>(mm) * p.N + n_base + col) = val;
+    }
+  }
+}
+
 template <int MP, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_swap_streamk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
@@ -1238,19 +1270,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           constexpr int ITER = SCALE_CAP / STEP;
           const int mm = tid % MP;
           const int v0 = chunk_base + tid / MP;
-          int vt = v0 / KB;
-          int vkb = v0 - vt * KB;
           float a[ITER], b[ITER];
+          // each unit's (tile, K block) is computed on its own, so that no load waits for an index
+          // chain: all of a thread's scale loads are in flight together
 #pragma unroll
           for (int r = 0; r < ITER; ++r) {
             a[r] = 0.0f;
             b[r] = 0.0f;
-            if (v0 + r * STEP < chunk_end) {
+            const int v = v0 + r * STEP;
+            if (v < chunk_end) {
+              const int vt = v / KB;
+              const int vkb = v - vt * KB;
               if (mm < p.M) a[r] = __ldg(p.sfa + static_cast<size_t>(vkb) * p.ld + mm);
               b[r] = __ldg(p.sfb + static_cast<size_t>(vt) * KB + vkb);
             }
-            vkb += STEP;
-            while (vkb >= KB) { vkb -= KB; ++vt; }
           }
 #pragma unroll
           for (int r = 0; r < ITER; ++r) s_scale[(tid / MP + r * STEP) * MP + mm] = a[r] * b[r];
@@ -1407,27 +1440,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     cluster_sync_all();  // every CTA's partial is in its shared memory
     if (warp < kPromoWarps && !*abort_flag) {
-      const int tid = threadIdx.x;
-      const int R4 = kBlockM / S / 4;  // float4 per token row of this CTA's slice
-      const int n_base = cl_tile * kBlockM;
-      const int rows = p.M < MP ? p.M : MP;
       const uint32_t part = smem_addr(smem);
-      for (int f = tid; f < rows * R4; f += NPROMO) {
-        const int mm = f / R4;
-        const int col = cl_rank * (kBlockM / S) + (f - mm * R4) * 4;
-        if (n_base + col < p.N) {  // N % 8 == 0, so the 4 columns are all inside
-          const uint32_t off = part + static_cast<uint32_t>((mm * kBlockM + col) * 4);
-          float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int q = 0; q < S; ++q) {
-            const float4 v = ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)));
-            r.x += v.x; r.y += v.y; r.z += v.z; r.w += v.w;
-          }
-          uint2 val;
-          val.x = pack_bf16x2(r.x, r.y);
-          val.y = pack_bf16x2(r.z, r.w);
-          *reinterpret_cast<uint2*>(p.C + static_cast<size_t>(mm) * p.N + n_base + col) = val;
-        }
-      }
+      const int n_base = cl_tile * kBlockM;
+      if (S == 2) cluster_reduce_store<2, MP>(p, part, cl_rank, n_base, threadIdx.x);
+      else if (S == 4) cluster_reduce_store<4, MP>(p, part, cl_rank, n_base, threadIdx.x);
+      else cluster_reduce_store<8, MP>(p, part, cl_rank, n_base, threadIdx.x);
     }
     __syncwarp();
     cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
