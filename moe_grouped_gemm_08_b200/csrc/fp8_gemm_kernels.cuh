@@ -49,7 +49,7 @@ constexpr int kMmaWarp = 9;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, far above any legal wait
 constexpr int kErrTimeout = 6;       // FG_ERR_TIMEOUT
 constexpr int kMaskedMaxGroups = 1024;
-constexpr int kSwapScaleBytes = 24 * 1024;  // shared memory for staged combined scales (swap kernel)
+constexpr int kSwapScaleBytes = 12 * 1024;  // shared memory for staged combined scales (swap kernel)
 constexpr int kSaChunk = 8;                 // K blocks per staged scale chunk (tiled kernel)
 constexpr int kTiledThreads = 384;          // tiled kernel: three warpgroups
 constexpr int kTiledLaunchRegs = 168;       // registers per thread the tiled kernel is launched with

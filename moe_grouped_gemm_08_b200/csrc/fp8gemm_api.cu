@@ -94,7 +94,7 @@ static_assert(pair_smem_bytes<kPairBN, kPairStages>() <= 227 * 1024, "pair kerne
 
 template <int MP>
 constexpr int swap_stages() {
-  return MP == 128 ? 5 : (MP == 64 ? 7 : 8);
+  return MP == 128 ? 5 : (MP == 64 ? 8 : 10);
 }
 
 template <int MP, int STAGES>
