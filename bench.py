@@ -243,6 +243,10 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is not None:
+            # a timed region shorter than nvidia-smi's start-up would otherwise end with no sample
+            deadline = time.time() + 3.0
+            while not self.samples and time.time() < deadline and self.proc.poll() is None:
+                time.sleep(0.02)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
