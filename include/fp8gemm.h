@@ -191,9 +191,10 @@ fg_status fg_get_device_status(void* stream);
 const char* fg_status_string(fg_status status);
 
 /* Kernel selection, process-wide: 0 = automatic (dense M <= 128 takes the
- * swap-AB stream-K kernel, everything else the one-CTA tiled kernel), 1 = the
- * one-CTA tiled kernel for every dense call, 2 = always swap-AB stream-K for
- * dense calls (requires M <= 128), 3 = the CTA-pair kernel (tcgen05 cta_group::2,
+ * swap-AB kernel, scheduled as fg_set_swap_schedule says, everything else the
+ * one-CTA tiled kernel), 1 = the one-CTA tiled kernel for every dense call, 2 =
+ * always the swap-AB kernel for dense calls (requires M <= 128), 3 = the CTA-pair
+ * kernel (tcgen05 cta_group::2,
  * 256-row tiles over two SMs) for dense and masked calls.  The contiguous layout
  * always takes the one-CTA tiled kernel.  Returns the previous value; an unknown
  * value is ignored. */

@@ -7,6 +7,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import moe_grouped_gemm_08_b200 as fg
 
@@ -47,6 +48,27 @@ def test_dense_path_switch():
     assert fg.set_dense_path(3) == 2
     assert fg.set_dense_path(7) == 3  # ignored
     fg.set_dense_path(old)
+
+
+def test_schedule_switches():
+    old = fg.set_swap_schedule(4)
+    assert old == 0  # automatic by default
+    assert fg.set_swap_schedule(-1) == 4
+    assert fg.set_swap_schedule(3) == -1  # not a cluster size: ignored
+    assert fg.set_swap_schedule(8) == -1
+    fg.set_swap_schedule(old)
+    old = fg.set_tiled_streamk(0)
+    assert old == 18  # default cost charged for publishing partial tiles, in K blocks
+    assert fg.set_tiled_streamk(-5) == 0
+    assert fg.set_tiled_streamk(old) == -1  # any negative value is stored as -1 (never split)
+
+
+def test_swap_plan_without_device_state():
+    # no fg_init on a machine without a GPU: the query answers -1 and launches nothing
+    if not torch.cuda.is_available():
+        assert fg.swap_plan(64, 2112, 7168) == -1
+    assert fg.swap_plan(0, 2112, 7168) == -1
+    assert fg.swap_plan(129, 2112, 7168) == -1
 
 
 NULL = None
