@@ -656,9 +656,9 @@ def main():
     ap.add_argument("--tiled-streamk", type=int, default=None, metavar="BLOCKS",
                     help="tiled kernel's stream-K tail threshold (fg_set_tiled_streamk): split the last "
                          "partial wave when it saves more than BLOCKS K blocks; negative: never")
-    ap.add_argument("--swap-schedule", type=int, default=None, choices=[-1, 0, 2, 4, 8],
+    ap.add_argument("--swap-schedule", type=int, default=None, choices=[-1, 0, 1, 2, 4, 8],
                     help="small-M kernel schedule (fg_set_swap_schedule): 0 automatic, -1 never the "
-                         "cluster split, 2/4/8 the cluster split with that many CTAs per tile")
+                         "cluster split, 1 whole tiles, 2/4/8 the cluster split with that many CTAs per tile")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

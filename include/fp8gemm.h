@@ -218,9 +218,10 @@ int fg_set_tiled_streamk(int overhead);
  * split: a thread-block cluster of S CTAs per weight tile, each CTA taking 1/S of the
  * K blocks, the partials summed through distributed shared memory (possible when every
  * tile's cluster can be resident at once and K has at least S blocks of 128); the
- * cheapest by a cost model in K blocks.  -1: never the cluster split.  2, 4 or 8: the
- * cluster split with that S wherever it is possible.  Other values are ignored.  All
- * schedules sum in a fixed order.  Returns the previous value. */
+ * cheapest by a cost model in K blocks.  -1: never the cluster split.  1: whole tiles,
+ * one CTA per tile up to the SM count.  2, 4 or 8: the cluster split with that S
+ * wherever it is possible.  Other values are ignored.  All schedules sum in a fixed
+ * order.  Returns the previous value. */
 int fg_set_swap_schedule(int schedule);
 
 /* The schedule the small-M kernel takes for a dense call of this shape on the current

@@ -126,8 +126,8 @@ def set_tiled_streamk(overhead: int) -> int:
 
 
 def set_swap_schedule(schedule: int) -> int:
-    """Small-M kernel schedule: 0 automatic, -1 never the cluster split, 2/4/8 the cluster split
-    with that many CTAs per weight tile wherever possible. Returns the old value."""
+    """Small-M kernel schedule: 0 automatic, -1 never the cluster split, 1 whole tiles, 2/4/8 the
+    cluster split with that many CTAs per weight tile wherever possible. Returns the old value."""
     return int(_lib.fg_set_swap_schedule(int(schedule)))
 
 

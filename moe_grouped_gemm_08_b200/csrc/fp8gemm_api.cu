@@ -434,7 +434,12 @@ SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
   if (c.tile_aligned) c.grid = sms;
   c.cluster = 1;
   const int sched = g_swap_schedule.load(std::memory_order_relaxed);
-  if (sched >= 0) {
+  if (sched == 1) {  // whole tiles, one CTA per tile up to the SM count
+    c.tile_aligned = 1;
+    c.grid = n_tiles < sms ? n_tiles : sms;
+    return c;
+  }
+  if (sched == 0 || sched > 1) {
     long long best = c.tile_aligned ? aligned_units : (split_units + (num_kb > 1 ? FG_SWAP_STREAMK_UNITS : 0));
     for (int S : {8, 4, 2}) {
       if (sched > 0 && S != sched) continue;
@@ -650,7 +655,7 @@ int fg_swap_plan(int M, int N, int K) {
 }
 
 int fg_set_swap_schedule(int schedule) {
-  if (schedule != 0 && schedule != -1 && schedule != 2 && schedule != 4 && schedule != 8)
+  if (schedule != 0 && schedule != -1 && schedule != 1 && schedule != 2 && schedule != 4 && schedule != 8)
     return g_swap_schedule.load();
   return g_swap_schedule.exchange(schedule);
 }

@@ -56,6 +56,7 @@ def test_schedule_switches():
     assert fg.set_swap_schedule(-1) == 4
     assert fg.set_swap_schedule(3) == -1  # not a cluster size: ignored
     assert fg.set_swap_schedule(8) == -1
+    assert fg.set_swap_schedule(1) == 8
     fg.set_swap_schedule(old)
     old = fg.set_tiled_streamk(0)
     assert old == 18  # default cost charged for publishing partial tiles, in K blocks
