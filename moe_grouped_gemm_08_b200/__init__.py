@@ -178,9 +178,24 @@ def _i32(t: torch.Tensor, what: str) -> torch.Tensor:
     return t
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device=None):
+    """The stream to launch on: ``stream``, or the current stream of ``device``; a given stream
+    must belong to ``device``."""
+    if stream is None:
+        s = torch.cuda.current_stream(device)
+    else:
+        s = stream
+        if device is not None and s.device != device:
+            raise ValueError(f"stream is on {s.device}, the operands on {device}")
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _same_device(device, **tensors):
+    """Every operand must live on the GPU the launch goes to (a pointer into another GPU's or into
+    host memory would be dereferenced by the kernel)."""
+    for name, t in tensors.items():
+        if t.device != device:
+            raise ValueError(f"{name} is on {t.device}, A on {device}")
 
 
 def _out(C, shape, device):
@@ -188,6 +203,8 @@ def _out(C, shape, device):
         return torch.empty(shape, dtype=torch.bfloat16, device=device)
     if C.dtype != torch.bfloat16 or tuple(C.shape) != tuple(shape) or not C.is_contiguous():
         raise ValueError(f"C must be a contiguous bfloat16 tensor of shape {tuple(shape)}")
+    if C.device != device:
+        raise ValueError(f"C is on {C.device}, the operands on {device}")
     return C
 
 
@@ -205,10 +222,13 @@ def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=
     if B.shape[1] != K or tuple(sfa.shape) != (_cdiv(K, 128), sfa_ld(M)) or \
             tuple(sfb.shape) != (_cdiv(N, 128), _cdiv(K, 128)):
         raise ValueError("inconsistent shapes")
-    C = _out(C, (M, N), A.device)
-    init(A.device.index)
-    _check(_lib.fp8_gemm_nt_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
-                               M, N, K, fa, fb, _stream(stream)), "fp8_gemm_nt")
+    dev = A.device
+    _same_device(dev, B=B, sfa=sfa, sfb=sfb)
+    C = _out(C, (M, N), dev)
+    with torch.cuda.device(dev):
+        init(dev.index)
+        _check(_lib.fp8_gemm_nt_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
+                                   M, N, K, fa, fb, _stream(stream, dev)), "fp8_gemm_nt")
     return C
 
 
@@ -222,11 +242,14 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None,
     if B.shape[2] != K or m_indices.numel() != M or tuple(sfa.shape) != (_cdiv(K, 128), sfa_ld(M)) or \
             tuple(sfb.shape) != (G, _cdiv(N, 128), _cdiv(K, 128)):
         raise ValueError("inconsistent shapes")
-    C = _out(C, (M, N), A.device)
-    init(A.device.index)
-    _check(_lib.fp8_gemm_grouped_contiguous_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                               C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb,
-                                               _stream(stream)), "fp8_gemm_grouped_contiguous")
+    dev = A.device
+    _same_device(dev, B=B, sfa=sfa, sfb=sfb, m_indices=m_indices)
+    C = _out(C, (M, N), dev)
+    with torch.cuda.device(dev):
+        init(dev.index)
+        _check(_lib.fp8_gemm_grouped_contiguous_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                                   C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb,
+                                                   _stream(stream, dev)), "fp8_gemm_grouped_contiguous")
     return C
 
 
@@ -240,11 +263,14 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stre
             tuple(sfa.shape) != (G, _cdiv(K, 128), sfa_ld(Mmax)) or \
             tuple(sfb.shape) != (G, _cdiv(N, 128), _cdiv(K, 128)):
         raise ValueError("inconsistent shapes")
-    C = _out(C, (G, Mmax, N), A.device)
-    init(A.device.index)
-    _check(_lib.fp8_gemm_grouped_masked_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                           C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb, _stream(stream)),
-           "fp8_gemm_grouped_masked")
+    dev = A.device
+    _same_device(dev, B=B, sfa=sfa, sfb=sfb, masked_m=masked_m)
+    C = _out(C, (G, Mmax, N), dev)
+    with torch.cuda.device(dev):
+        init(dev.index)
+        _check(_lib.fp8_gemm_grouped_masked_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                               C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb,
+                                               _stream(stream, dev)), "fp8_gemm_grouped_masked")
     return C
 
 
@@ -264,8 +290,9 @@ def cast_fp8_rows(x, stream=None, fmt="e4m3"):
     G, M, K = (x.shape if grouped else (1,) + tuple(x.shape))
     q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     sfa = torch.zeros((G, _cdiv(K, 128), sfa_ld(M)), dtype=torch.float32, device=x.device)
-    _check(_lib.fp8_cast_rows_ex(x.data_ptr(), q.data_ptr(), sfa.data_ptr(), G, M, K, FORMATS[fmt],
-                                 _stream(stream)), "fp8_cast_rows")
+    with torch.cuda.device(x.device):
+        _check(_lib.fp8_cast_rows_ex(x.data_ptr(), q.data_ptr(), sfa.data_ptr(), G, M, K, FORMATS[fmt],
+                                     _stream(stream, x.device)), "fp8_cast_rows")
     return q, (sfa if grouped else sfa[0])
 
 
@@ -277,6 +304,7 @@ def cast_fp8_blocks(w, stream=None, fmt="e4m3"):
     G, N, K = (w.shape if grouped else (1,) + tuple(w.shape))
     q = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
     sfb = torch.empty((G, _cdiv(N, 128), _cdiv(K, 128)), dtype=torch.float32, device=w.device)
-    _check(_lib.fp8_cast_blocks_ex(w.data_ptr(), q.data_ptr(), sfb.data_ptr(), G, N, K, FORMATS[fmt],
-                                   _stream(stream)), "fp8_cast_blocks")
+    with torch.cuda.device(w.device):
+        _check(_lib.fp8_cast_blocks_ex(w.data_ptr(), q.data_ptr(), sfb.data_ptr(), G, N, K, FORMATS[fmt],
+                                       _stream(stream, w.device)), "fp8_cast_blocks")
     return q, (sfb if grouped else sfb[0])

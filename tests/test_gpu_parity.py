@@ -237,3 +237,23 @@ def _masked_counts_edge_cases(fg):
 
 def test_device_status_clean(fg):
     assert fg.device_status() == 0
+
+
+def test_output_in_host_memory_is_rejected(fg):
+    """A host-memory output is refused before any launch, for all three layouts."""
+    case = synth.dense_case(7, 64, 256, 256)
+    A, sfa, B, sfb = dense_dev(case)
+    before = fg.launch_count()
+    with pytest.raises(ValueError):
+        fg.gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=torch.empty((64, 256), dtype=torch.bfloat16))
+    cc = synth.contiguous_case(8, [64, 64], N=136, K=256)
+    with pytest.raises(ValueError):
+        fg.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(to_dev(cc["A"]), to_dev(cc["sfa"]), to_dev(cc["B"]),
+                                                     to_dev(cc["sfb"]), to_dev(cc["m_indices"]),
+                                                     C=torch.empty((cc["M"], cc["N"]), dtype=torch.bfloat16))
+    mc = synth.masked_case(9, 2, 128, 136, 256, masked_m=[5, 128])
+    with pytest.raises(ValueError):
+        fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(to_dev(mc["A"]), to_dev(mc["sfa"]), to_dev(mc["B"]),
+                                                 to_dev(mc["sfb"]), to_dev(mc["masked_m"]),
+                                                 C=torch.empty((2, 128, 136), dtype=torch.bfloat16))
+    assert fg.launch_count() == before
