@@ -112,6 +112,12 @@ static const double *dec_table_fmt(int fmt) {
     return g_dec52;
 }
 
+/* Build both decode tables before a parallel region (they are filled lazily, once). */
+static void tables_ready(void) {
+    (void)dec_table();
+    (void)dec_table_fmt(1);
+}
+
 void oracle_e5m2_decode_table(double *out256) {
     memcpy(out256, dec_table_fmt(1), 256 * sizeof(double));
 }
@@ -124,7 +130,7 @@ static int quantum_exp(int fmt) { return fmt == 0 ? 9 : 16; }
 
 static int64_t code_units(int fmt, uint8_t code) {
     double v = dec_table_fmt(fmt)[code];
-    if (!isfinite(v)) return 0;  /* inputs are finite */
+    if (!isfinite(v)) return 0;  /* non-finite codes take the fp64 path in row_nt */
     return (int64_t)ldexp(v, quantum_exp(fmt));
 }
 
@@ -168,6 +174,7 @@ static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
                    const uint8_t *B, const float *sfb, int N, int K,
                    uint16_t *c_row, double *acc_row, int fa, int fb) {
     const double *dec = dec_table();
+    const double *deca = dec_table_fmt(fa), *decb = dec_table_fmt(fb);
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     int64_t ua[256], ub[256];
     if (fa != 0 || fb != 0)
@@ -182,9 +189,19 @@ static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
             if (fa == 0 && fb == 0) {
                 for (int k = k0; k < k1; ++k) s += dec[a_row[k]] * dec[b_row[k]];
             } else {
-                __int128 t = 0;
-                for (int k = k0; k < k1; ++k) t += (__int128)ua[a_row[k]] * ub[b_row[k]];
-                s = ldexp((double)t, -(quantum_exp(fa) + quantum_exp(fb)));
+                /* a block holding a non-finite code (e4m3 NaN; e5m2 infinity or NaN) is summed in
+                 * fp64: the IEEE result (NaN, or an infinity) does not depend on the finite terms'
+                 * rounding; every other block exactly, in quanta */
+                int special = 0;
+                for (int k = k0; k < k1 && !special; ++k)
+                    special = !isfinite(deca[a_row[k]]) || !isfinite(decb[b_row[k]]);
+                if (special) {
+                    for (int k = k0; k < k1; ++k) s += deca[a_row[k]] * decb[b_row[k]];
+                } else {
+                    __int128 t = 0;
+                    for (int k = k0; k < k1; ++k) t += (__int128)ua[a_row[k]] * ub[b_row[k]];
+                    s = ldexp((double)t, -(quantum_exp(fa) + quantum_exp(fb)));
+                }
             }
             double scale = (double)sfa_m[(size_t)kb * ld] *
                            (double)sfb[(size_t)(n / ORC_BLOCK) * KB + kb];
@@ -200,6 +217,7 @@ static void row_nt(const uint8_t *a_row, const float *sfa_m, long ld,
 void oracle_gemm_nt(const uint8_t *A, const float *sfa, long ld,
                     const uint8_t *B, const float *sfb,
                     int M, int N, int K, uint16_t *C, double *acc, int fa, int fb) {
+    tables_ready();
     #pragma omp parallel for schedule(dynamic, 1)
     for (int m = 0; m < M; ++m)
         row_nt(A + (size_t)m * K, sfa + m, ld, B, sfb, N, K,
@@ -213,6 +231,7 @@ void oracle_gemm_nt_rows(const uint8_t *A, const float *sfa, long ld,
                          int M, int N, int K, const int *rows, int nrows,
                          uint16_t *C, double *acc, int fa, int fb) {
     (void)M;
+    tables_ready();
     #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < nrows; ++i) {
         int m = rows[i];
@@ -236,6 +255,7 @@ void oracle_grouped_contiguous(const uint8_t *A, const float *sfa, long ld,
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
     int count = rows ? nrows : M_total;
+    tables_ready();
     #pragma omp parallel for schedule(dynamic, 1)
     for (int i = 0; i < count; ++i) {
         int m = rows ? rows[i] : i;
@@ -258,6 +278,7 @@ void oracle_grouped_masked(const uint8_t *A, const float *sfa, long ld,
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
     long total = (long)G * Mmax;
+    tables_ready();
     #pragma omp parallel for schedule(dynamic, 1)
     for (long gm = 0; gm < total; ++gm) {
         int g = (int)(gm / Mmax);
@@ -357,6 +378,7 @@ static float block_scale(float amax, int fmt) {
 void oracle_quantize_rows(const uint16_t *X, int G, int M, int K, uint8_t *Q, float *sfa, long ld, int fmt) {
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     long rows = (long)G * M;
+    tables_ready();
     #pragma omp parallel for schedule(static)
     for (long r = 0; r < rows; ++r) {
         const int g = (int)(r / M), m = (int)(r % M);
@@ -384,6 +406,7 @@ void oracle_quantize_blocks(const uint16_t *X, int G, int N, int K, uint8_t *Q, 
     const int KB = (K + ORC_BLOCK - 1) / ORC_BLOCK;
     const int NB = (N + ORC_BLOCK - 1) / ORC_BLOCK;
     long blocks = (long)G * NB * KB;
+    tables_ready();
     #pragma omp parallel for schedule(static)
     for (long b = 0; b < blocks; ++b) {
         const int g = (int)(b / ((long)NB * KB));

@@ -177,3 +177,47 @@ def test_e5m2_pins_catch_planted_mistake(name, tmp_path):
     finally:
         oracle._LIB = saved
     assert caught, f"no pin caught the planted mistake {name!r}"
+
+
+# ---------------------------------------------------------------------------- non-finite codes
+from tests import test_oracle_specials as special_pins  # noqa: E402
+
+SPECIAL_MUTANTS = {
+    # non-finite codes counted as zero in the exact integer sums
+    "specials_dropped": ("special = !isfinite(deca[a_row[k]]) || !isfinite(decb[b_row[k]]);", "special = 0;"),
+    # a special block summed with the finite codes only
+    "specials_skipped": ("for (int k = k0; k < k1; ++k) s += deca[a_row[k]] * decb[b_row[k]];",
+                         "for (int k = k0; k < k1; ++k) if (isfinite(deca[a_row[k]] * decb[b_row[k]])) "
+                         "s += deca[a_row[k]] * decb[b_row[k]];"),
+}
+
+SPECIAL_PINS = [
+    lambda: [special_pins.test_nan_code_in_a_poisons_its_row(fa, fb, 0x7F)
+             for fa, fb in [("e5m2", "e5m2"), ("e4m3", "e5m2")]],
+    lambda: special_pins.test_e5m2_infinity_keeps_the_sign_of_the_product("e5m2"),
+    special_pins.test_opposite_infinities_in_one_sum_give_nan,
+    lambda: special_pins.test_every_e5m2_nan_code_propagates(0x7E),
+]
+
+
+@pytest.mark.parametrize("name", sorted(SPECIAL_MUTANTS))
+def test_special_pins_catch_planted_mistake(name, tmp_path):
+    before, after = SPECIAL_MUTANTS[name]
+    text = SRC.read_text()
+    assert text.count(before) == 1, name
+    (tmp_path / "m.c").write_text(text.replace(before, after))
+    so = tmp_path / f"liboracle_{name}.so"
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fopenmp", "-fPIC",
+                           "-shared", str(tmp_path / "m.c"), "-o", str(so), "-lm"])
+    saved = oracle._lib()
+    oracle._LIB = oracle.load(so)
+    caught = 0
+    try:
+        for pin in SPECIAL_PINS:
+            try:
+                pin()
+            except AssertionError:
+                caught += 1
+    finally:
+        oracle._LIB = saved
+    assert caught, f"no pin caught the planted mistake {name!r}"
