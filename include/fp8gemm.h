@@ -162,7 +162,8 @@ fg_status fg_noalloc_status(void* stream);
  *   code  = e4m3 round-to-nearest-even of the fp32 quotient x / scale, saturating
  *           at +-448,
  * so that dec(code) * scale approximates x.  Results are exact and deterministic
- * (no accumulation).  K % 16 == 0; X and Q 16-byte aligned, scales 4-byte aligned;
+ * (no accumulation).  X must be finite: a block holding an infinity or a NaN gets
+ * unspecified codes and scale.  K % 16 == 0; X and Q 16-byte aligned, scales 4-byte aligned;
  * all pointers are device pointers owned by the caller; nothing is allocated.
  *
  * fp8_cast_rows: the A side (activations).  X is [G][M][K] (G = 1 for a plain
