@@ -77,15 +77,16 @@ def load_traffic(kernel: str, workload: str):
     return entry
 
 
-def record_traffic(csv_path: str, workload: str) -> None:
+def record_traffic(csv_path: str, workload: str, out_path: str | None = None) -> None:
     """Average dram__bytes_read.sum + dram__bytes_write.sum per launch of each of this library's
-    kernels in an ncu --csv launch list, stored in profiles/traffic.json with the kernel source hash."""
+    kernels in an ncu --csv launch list, stored (default: profiles/traffic.json) with the kernel
+    source hash."""
     import csv as _csv
     rows = [r for r in _csv.reader(open(csv_path)) if r]
     hi = next(i for i, r in enumerate(rows) if "Kernel Name" in r and "Metric Name" in r)
     h = rows[hi]
     col = {k: h.index(k) for k in ("ID", "Kernel Name", "Metric Name", "Metric Unit", "Metric Value")}
-    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+    scale = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
     per = {}
     for r in rows[hi + 1:]:
         if len(r) != len(h) or not r[col["Metric Name"]].startswith("dram__bytes_"):
@@ -95,10 +96,13 @@ def record_traffic(csv_path: str, workload: str) -> None:
                      if k in name), None)
         if kern is None:
             continue
-        v = float(r[col["Metric Value"]].replace(",", "")) * scale.get(r[col["Metric Unit"]], 1)
+        unit = r[col["Metric Unit"]]
+        if unit not in scale:
+            raise ValueError(f"unexpected unit {unit!r} for {r[col['Metric Name']]}")
+        v = float(r[col["Metric Value"]].replace(",", "")) * scale[unit]
         per.setdefault(kern, {}).setdefault(r[col["ID"]], 0.0)
         per[kern][r[col["ID"]]] += v
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = out_path or os.path.join(ROOT, "profiles", "traffic.json")
     d = json.load(open(path)) if os.path.exists(path) else {}
     for kern, launches in per.items():
         d[f"{kern}:{workload}"] = {"dram_bytes_per_launch": round(sum(launches.values()) / len(launches)),
@@ -138,7 +142,7 @@ def work_of(case):
     N, K = case["N"], case["K"]
     KB, NB = cdiv(K, 128), cdiv(N, 128)
     if case["kind"] == "masked":
-        valid = np.minimum(case["masked_m"], case["Mmax"]).astype(np.int64)
+        valid = np.clip(np.asarray(case["masked_m"], dtype=np.int64), 0, case["Mmax"])  # as the kernel reads it
         Mv = int(valid.sum())
         groups_used = int((valid > 0).sum())
         G = case["G"]
@@ -147,11 +151,13 @@ def work_of(case):
         pages = G * case["Mmax"] * K + G * N * K + 2 * G * case["Mmax"] * N
         return flops, byt, pages
     if case["kind"] == "contiguous":
-        Mv = int((case["m_indices"] >= 0).sum())
-        G = case["G"]
+        mi = np.asarray(case["m_indices"])
+        live = (mi >= 0) & (mi < case["G"])  # indices >= G are padding, as in the kernel
+        Mv = int(live.sum())
+        groups_used = int(np.unique(mi[live]).size)  # B is needed only for groups with a valid row
         flops = 2 * Mv * N * K
-        byt = Mv * K + G * N * K + 2 * Mv * N + 4 * Mv * KB + 4 * G * NB * KB
-        return flops, byt, Mv * K + G * N * K + 2 * Mv * N
+        byt = Mv * K + groups_used * N * K + 2 * Mv * N + 4 * Mv * KB + 4 * groups_used * NB * KB
+        return flops, byt, Mv * K + groups_used * N * K + 2 * Mv * N
     M = case["M"]
     flops = 2 * M * N * K
     byt = M * K + N * K + 2 * M * N + 4 * M * KB + 4 * NB * KB
