@@ -3,9 +3,14 @@
 
 One step = one pass of the chosen workload (default: the dense decode sweep, M in
 {64,128} x six (N,K) DeepSeek-V3/R1 shapes = 12 GEMM launches) over inputs
-already resident in HBM.  Prints ONE JSON line on rank 0.
+already resident in HBM.  Prints ONE JSON line on rank 0.  The headline keys
+(value, roofline, e2e, cpu_baseline) are the decode sweep's; the other four
+configurations (dense 128x256x512, prefill M=4096, contiguous, masked) are timed
+the same way in the same run, with the same steps and warm-up, and reported under
+"workloads" (--also selects them).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--also LIST]
+                  [--impl ours|reference]
 
 Timing: each step is replayed from a CUDA graph (the masked-layout call is made
 for graphs; the dense calls are captured the same way so that host launch cost
@@ -445,20 +450,10 @@ def run_cast(args, rank, world, local):
 
 
 # ---------------------------------------------------------------------------- our arm
-def run_ours(args, rank, world, local):
-    import moe_grouped_gemm_08_b200 as fg
-
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    fg.init(local)
-    global KERNEL_PATH
-    KERNEL_PATH = args.path
-    fg.set_dense_path(args.path)
-    if args.tiled_streamk is not None:
-        fg.set_tiled_streamk(args.tiled_streamk)
-    if args.swap_schedule is not None:
-        fg.set_swap_schedule(args.swap_schedule)
-    name, wl = workload_list(args.workload, args.shape)
+def measure_workload(fg, name, wl, args, dev, stream, world, local):
+    """Time one workload: each step (one call per GEMM of the workload) is replayed from a CUDA
+    graph, inputs rotating over enough copies that every launch reads HBM.  Returns the workload's
+    result dict, its cases and the device copies (for the end-to-end leg)."""
     cases = [make_case(w) for w in wl]
     works = [work_of(c) for c in cases]
     step_flops = sum(w[0] for w in works)
@@ -468,7 +463,6 @@ def run_ours(args, rank, world, local):
     # rotation: enough input copies that one copy is re-read only after > 3x L2 of other traffic
     rot = max(2, min(8, cdiv(3 * L2_BYTES, max(1, step_in_bytes)) + 1))
     devs = [[upload(c, dev) for c in cases] for _ in range(rot)]
-    stream = torch.cuda.Stream(device=dev)
 
     # eager warm-up call per case (sets kernel attributes before capture), then capture one graph per copy
     with torch.cuda.stream(stream):
@@ -532,13 +526,15 @@ def run_ours(args, rank, world, local):
             for i in range(len(cases)):
                 per_case_ms[i].append(evs[i].elapsed_time(evs[i + 1]))
     status = fg.device_status(stream)
+    del graphs, egraphs
 
     total_flops = step_flops * args.steps * world
     value = total_flops / (elapsed_ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
     shapes = []
-    sum_bytes_swap, sum_ms_swap, sum_ms_all = 0.0, 0.0, 0.0
+    sum_bytes_dom, sum_ms_dom, sum_ms_all = 0.0, 0.0, 0.0
+    dom = kernel_name(cases[0])
     for c, w, wk, ts in zip(cases, wl, works, per_case_ms):
         ms = statistics.mean(ts)
         tfl = wk[0] / (ms * 1e-3) / 1e12
@@ -552,34 +548,64 @@ def run_ours(args, rank, world, local):
             plan = fg.swap_plan(c["M"], c["N"], c["K"])
             shapes[-1]["schedule"] = {0: "stream-K", 1: "whole tiles"}.get(plan, f"cluster x{plan}")
         sum_ms_all += ms
-        if kernel_name(c) == kernel_name(cases[0]):
-            sum_bytes_swap += wk[1]
-            sum_ms_swap += ms
-    dom = kernel_name(cases[0])
-    dom_bound = "hbm" if all(s["bound"] == "hbm" for s in shapes if s["kernel"] == dom) else "tensor"
+        if kernel_name(c) == dom:
+            sum_bytes_dom += wk[1]
+            sum_ms_dom += ms
+    # the roofline's bound is the one of the dominant kernel's work taken together
+    dom_flops = sum(wk[0] for c, wk in zip(cases, works) if kernel_name(c) == dom)
+    dom_bound = "hbm" if sum_bytes_dom / (peaks["hbm_gbs"] * 1e9) > dom_flops / (fp8_peak * 1e12) else "tensor"
     single_kernel = all(kernel_name(c) == dom for c in cases)
     if single_kernel:
         # every launch of the timed region is this kernel: its average launch duration is the
         # timed region divided by the launches (inter-kernel gaps included)
-        sum_ms_swap = elapsed_ms / args.steps
-        sum_ms_all = sum_ms_swap
+        sum_ms_dom = elapsed_ms / args.steps
+        sum_ms_all = sum_ms_dom
     if dom_bound == "hbm":
-        achieved = sum_bytes_swap / (sum_ms_swap * 1e-3) / 1e9
+        achieved = sum_bytes_dom / (sum_ms_dom * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4)}
     else:
-        dom_flops = sum(wk[0] for c, wk in zip(cases, works) if kernel_name(c) == dom)
-        achieved = dom_flops / (sum_ms_swap * 1e-3) / 1e12
+        achieved = dom_flops / (sum_ms_dom * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp8_peak, 1), "unit": "TFLOP/s",
                 "frac": round(achieved / fp8_peak, 4)}
     tr = load_traffic(dom, name)
     roof["traffic"] = tr["dram_bytes_per_launch"] if tr else None
     roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if dom_bound == 'hbm' else 'bf16_tflops x 2 nominal fp8/bf16'})"
     roof["kernel"] = dom
-    roof["launch_share"] = round(sum_ms_swap / sum_ms_all, 4) if sum_ms_all else None
+    roof["launch_share"] = round(sum_ms_dom / sum_ms_all, 4) if sum_ms_all else None
+    roof["algorithmic_bytes_per_step"] = int(sum_bytes_dom)
+    roof["algorithmic_flops_per_step"] = int(dom_flops)
     roof["bytes_per_launch_def"] = "A + B + C + fp32 scales, valid rows, per launch; summed over the step"
     roof["timing"] = ("timed region / launches" if single_kernel else
                       "event-instrumented pass after the timed region")
+    res = {"value": round(value, 2), "unit": "TFLOPS", "ms_per_step": round(elapsed_ms / args.steps, 5),
+           "steps": args.steps, "warmup": args.warmup,
+           "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
+           "config": {"workload": name, "shapes": [w["name"] for w in wl],
+                      "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
+                      "graph": "each step replayed from a CUDA graph"},
+           "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
+           "roofline": roof, "gpu_launches": launches_per_step * args.steps,
+           "clocks": clocks.summary(t_wall0, t_wall1), "device_status": fg.STATUS_NAMES.get(status, status)}
+    return res, cases, devs, step_flops
+
+
+def run_ours(args, rank, world, local):
+    import moe_grouped_gemm_08_b200 as fg
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fg.init(local)
+    global KERNEL_PATH
+    KERNEL_PATH = args.path
+    fg.set_dense_path(args.path)
+    if args.tiled_streamk is not None:
+        fg.set_tiled_streamk(args.tiled_streamk)
+    if args.swap_schedule is not None:
+        fg.set_swap_schedule(args.swap_schedule)
+    stream = torch.cuda.Stream(device=dev)
+    name, wl = workload_list(args.workload, args.shape)
+    res, cases, devs, step_flops = measure_workload(fg, name, wl, args, dev, stream, world, local)
 
     # end to end through the public API with host buffers: H2D of the step's inputs, GEMMs, D2H of C
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -617,29 +643,37 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
     barrier(world, local)
     e2e_value = step_flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
+    del host, outs, devs
 
-    line = {"metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 5), "higher_is_better": True,
+    line = {"metric": METRIC, "value": res["value"], "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3 (fp32 accumulate, bf16 out)",
             "data": "synthetic",
-            "config": {"workload": name, "shapes": [w["name"] for w in wl],
-                       "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
-                       "graph": "each step replayed from a CUDA graph", "parallelism": f"replicas x{world}",
-                       "kernel_path": args.path,
-                       "tiled_streamk": "library default" if args.tiled_streamk is None else args.tiled_streamk,
-                       "swap_schedule": "library default" if args.swap_schedule is None else args.swap_schedule},
-            "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
-            "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
-            "roofline": roof,
+            "config": dict(res["config"], parallelism=f"replicas x{world}", kernel_path=args.path,
+                           tiled_streamk="library default" if args.tiled_streamk is None else args.tiled_streamk,
+                           swap_schedule="library default" if args.swap_schedule is None else args.swap_schedule),
+            "hbm_gbs": res["hbm_gbs"], "shapes": res["shapes"], "shapes_timing": res["shapes_timing"],
+            "roofline": res["roofline"],
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": launches_per_step * args.steps,
-            "clocks": clocks.summary(t_wall0, t_wall1), "device_status": fg.STATUS_NAMES.get(status, status)}
+            "gpu_launches": res["gpu_launches"], "clocks": res["clocks"], "device_status": res["device_status"]}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         s, f, cores = time_oracle(cases, row_fraction=1.0)
         line["cpu_baseline"] = {"value": round(f / s / 1e12, 5), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                                 "sample": f"one full step of the {name} workload (every GEMM, all rows), {s:.1f} s"}
-    del graphs, egraphs
+    del cases
+    torch.cuda.empty_cache()
+
+    # the other configurations, timed the same way in the same process (same steps and warm-up)
+    extra = [x for x in (args.also.split(",") if args.also else []) if x and x != name]
+    if extra and not args.shape:
+        line["workloads"] = {}
+        for other in extra:
+            oname, owl = workload_list(other)
+            ores, ocases, odevs, _ = measure_workload(fg, oname, owl, args, dev, stream, world, local)
+            del ocases, odevs
+            torch.cuda.empty_cache()
+            line["workloads"][oname] = ores
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -653,6 +687,9 @@ def main():
                     help="decode_sweep (default), dense_single, prefill, contiguous, masked, or cast (the bf16 -> "
                          "e4m3 cast of the prefill operands)")
     ap.add_argument("--shape", default=None, help="M,N,K: one dense GEMM instead of a workload (profiling)")
+    ap.add_argument("--also", default="dense_single,prefill,contiguous,masked",
+                    help="comma-separated workloads timed after the headline one in the same run, reported "
+                         "under the 'workloads' key (empty: none)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")

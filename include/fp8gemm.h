@@ -232,12 +232,13 @@ int fg_set_swap_schedule(int schedule);
 int fg_swap_plan(int M, int N, int K);
 
 /* Failure injection for tests (process-wide, default 0).  With 1, every kernel of
- * fp8_gemm_nt that takes the small-M (swap-AB stream-K) path first waits on a barrier
- * that no one arrives at; the bounded wait runs out after about two seconds, the
- * kernel aborts cleanly (its other warps leave their waits, copies in flight are
- * drained, TMEM is freed), writes no output and leaves FG_ERR_TIMEOUT in the device
- * status word for fg_get_device_status().  Nothing faults or traps, and the context
- * stays usable.  Returns the previous value.  Not for production use. */
+ * fp8_gemm_nt that takes the small-M (swap-AB stream-K) path, and every kernel of
+ * fp8_gemm_nt_noalloc, first waits on a barrier that no one arrives at; the bounded
+ * wait runs out after about two seconds, the kernel aborts cleanly (its other warps
+ * leave their waits, copies in flight are drained, TMEM is freed), writes no output
+ * and leaves FG_ERR_TIMEOUT in the device status word for fg_get_device_status()
+ * (fg_noalloc_status() for the allocation-free variant).  Nothing faults or traps,
+ * and the context stays usable.  Returns the previous value.  Not for production use. */
 int fg_debug_set_stall(int enable);
 
 /* Number of GEMM kernel launches the library has issued in this process. */

@@ -503,32 +503,36 @@ constexpr size_t kNoAllocBytes = kNoAllocPartialBytes + kNoAllocCounters * sizeo
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
 
 struct NoAllocDevice {
-  bool ready = false;
+  std::atomic<bool> ready{false};  // published (release) after sms and base are set
   int sms = 0;
   unsigned char* base = nullptr;  // device address of g_noalloc_scratch on this device
 };
 NoAllocDevice g_noalloc[kMaxDevices];
 
 fg_status noalloc_setup(int dev, NoAllocDevice** out) {
-  std::lock_guard<std::mutex> lock(g_mutex);
   NoAllocDevice& d = g_noalloc[dev];
-  if (!d.ready) {
-    if (!g_encode) {
-      void* fn = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-          q != cudaDriverEntryPointSuccess || fn == nullptr)
+  if (!d.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!d.ready.load(std::memory_order_relaxed)) {
+      if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+          return FG_ERR_CUDA;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+      int major = 0, minor = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
         return FG_ERR_CUDA;
-      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      if (major != 10 || minor != 0) return FG_ERR_UNSUPPORTED;  // built for sm_100a only, as fg_init
+      if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FG_ERR_CUDA;
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FG_ERR_CUDA;
+      d.base = static_cast<unsigned char*>(ptr);
+      d.ready.store(true, std::memory_order_release);
     }
-    int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return FG_ERR_CUDA;
-    if (major != 10) return FG_ERR_UNSUPPORTED;
-    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FG_ERR_CUDA;
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FG_ERR_CUDA;
-    d.base = static_cast<unsigned char*>(ptr);
-    d.ready = true;
   }
   *out = &d;
   return FG_OK;
@@ -551,7 +555,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.ld = fg_sfa_ld(M);
   p.num_kb = (K + kBlockK - 1) / kBlockK;
   p.n_tiles = (N + kBlockM - 1) / kBlockM;
-  p.debug_stall = 0;
+  p.debug_stall = g_debug_stall.load(std::memory_order_relaxed);
   p.fmt_bits = 0;  // e4m3 x e4m3
   p.tile_aligned = 0;
   p.cluster = 1;
@@ -763,7 +767,8 @@ fg_status fp8_gemm_nt_noalloc(const void* A, const float* sfa, const void* B, co
 
 fg_status fg_noalloc_status(void* stream) {
   const int dev = current_device();
-  if (dev < 0 || dev >= kMaxDevices || !g_noalloc[dev].ready) return FG_OK;  // never called here
+  if (dev < 0 || dev >= kMaxDevices || !g_noalloc[dev].ready.load(std::memory_order_acquire))
+    return FG_OK;  // never called here
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FG_ERR_CUDA;
   int* status = reinterpret_cast<int*>(g_noalloc[dev].base + kNoAllocPartialBytes) + kNoAllocCounters;
   int v = 0;

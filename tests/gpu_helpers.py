@@ -53,3 +53,22 @@ def close(c_bits: np.ndarray, r_bits: np.ndarray, what: str = "") -> dict:
 
 def dense_dev(case):
     return (to_dev(case["A"]), to_dev(case["sfa"]), to_dev(case["B"]), to_dev(case["sfb"]))
+
+
+def close_nonfinite(c_bits: np.ndarray, r_bits: np.ndarray, what: str = "") -> dict:
+    """For outputs that non-finite input codes reach: NaN exactly where the oracle has NaN, the same
+    signed infinity where it has one, and the finite rest within the stated tolerance."""
+    c = oracle.bf16_bits_to_f32(c_bits).astype(np.float64)
+    r = oracle.bf16_bits_to_f32(r_bits).astype(np.float64)
+    assert c.shape == r.shape, (c.shape, r.shape)
+    nan_c, nan_r = np.isnan(c), np.isnan(r)
+    if not np.array_equal(nan_c, nan_r):
+        bad = np.argwhere(nan_c != nan_r)[:5]
+        raise AssertionError(f"{what}: NaN positions differ, e.g. at {bad.tolist()}")
+    inf_r = np.isinf(r)
+    if not np.array_equal(np.isinf(c), inf_r) or not np.array_equal(c[inf_r], r[inf_r]):
+        bad = np.argwhere((np.isinf(c) != inf_r) | (inf_r & (c != r)))[:5]
+        raise AssertionError(f"{what}: infinities differ, e.g. at {bad.tolist()}")
+    fin = ~(nan_r | inf_r)
+    stats = close(c_bits[fin], r_bits[fin], what) if fin.any() else {}
+    return dict(stats, nan=int(nan_r.sum()), inf=int(inf_r.sum()))
