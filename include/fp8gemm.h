@@ -38,10 +38,12 @@
  *
  * Ownership: the caller owns every buffer.  The library allocates only in
  * fg_init (a status word, a split-K workspace and its counters), never inside
- * a GEMM call, so calls can be captured into CUDA graphs.  The workspace is
- * per device and every GEMM entry point may use it (split tiles of the small-M
- * kernel and of the tiled kernel's last wave), so GEMM calls must not run
- * concurrently on different streams of the same device.
+ * a GEMM call, so calls can be captured into CUDA graphs.  The library's
+ * workspace is per device and every GEMM entry point may use it (split tiles of
+ * the small-M kernel and of the tiled kernel's last wave), so calls that use it
+ * must not run concurrently on different streams of the same device; the _ws
+ * entry points take a caller-owned workspace instead (one per stream lets
+ * GEMMs run concurrently on several streams).
  *
  * Errors: every entry point returns a status code and never throws.  Argument
  * errors are found on the host before any launch and launch nothing.  A device
@@ -51,6 +53,7 @@
 #ifndef FP8GEMM_H
 #define FP8GEMM_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -64,7 +67,11 @@ typedef enum {
   FG_ERR_UNSUPPORTED = 3,     /* valid but outside what this build supports (e.g. G > 1024) */
   FG_ERR_NOT_INITIALIZED = 4, /* fg_init was not called for the current device */
   FG_ERR_CUDA = 5,            /* a CUDA runtime / driver call failed */
-  FG_ERR_TIMEOUT = 6          /* a device-side wait ran out; the kernel exited early */
+  FG_ERR_TIMEOUT = 6,         /* a device-side wait ran out; the kernel exited early */
+  FG_ERR_DEVICE_CHECK = 7     /* debug build only: a device-side index check failed (an expert index
+                                 in m_indices outside [-1, G), a TMA tile coordinate outside its
+                                 tensor, a split-K workspace slot or counter out of range); the
+                                 kernel finished as a release build would */
 } fg_status;
 
 /* FP8 operand formats (the aisharenet.com how-to, "Main functions": the FP8 inputs
@@ -128,6 +135,32 @@ fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void
                                      void* C, const int* masked_m, int G, int Mmax, int N, int K,
                                      int fmt_a, int fmt_b, void* stream);
 
+/* Size in bytes of a caller-owned split-K workspace for the current device (it depends on
+ * the SM count): two fp32 partial tiles of 128 x 256 per SM, then 65536 int32 counters.
+ * 0 if fg_init was not called for the device. */
+size_t fg_workspace_bytes(void);
+
+/* The three GEMMs with a caller-owned workspace (device memory, 16-byte aligned, at least
+ * fg_workspace_bytes() bytes, zero-filled once before its first use, e.g. with
+ * cudaMemsetAsync).  Every kernel leaves the counters at zero again when it finishes, so
+ * a workspace can be reused by any number of calls in stream order; calls that may run
+ * at the same time (different streams) need different workspaces.  After a call ends
+ * with FG_ERR_TIMEOUT (fg_get_device_status) the caller zero-fills its workspace again.
+ * workspace == NULL with workspace_bytes == 0 uses the library's own workspace (the _ex
+ * entry points); a workspace that is too small is FG_ERR_INVALID_ARG, a misaligned one
+ * FG_ERR_ALIGNMENT.  Everything else is as for the _ex entry points. */
+fg_status fp8_gemm_nt_ws(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                         int M, int N, int K, int fmt_a, int fmt_b, void* workspace,
+                         size_t workspace_bytes, void* stream);
+fg_status fp8_gemm_grouped_contiguous_ws(const void* A, const float* sfa, const void* B, const float* sfb,
+                                         void* C, const int* m_indices, int M_total, int G, int N, int K,
+                                         int fmt_a, int fmt_b, void* workspace, size_t workspace_bytes,
+                                         void* stream);
+fg_status fp8_gemm_grouped_masked_ws(const void* A, const float* sfa, const void* B, const float* sfb,
+                                     void* C, const int* masked_m, int G, int Mmax, int N, int K,
+                                     int fmt_a, int fmt_b, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
 /* Allocation-free variant of fp8_gemm_nt, for callers that cannot allocate device
  * memory: code running inside another framework's memory pool or a pre-planned
  * static memory budget, code that must not touch the allocator during a
@@ -185,7 +218,9 @@ fg_status fp8_cast_rows_ex(const void* X, void* Q, float* sfa, int G, int M, int
 fg_status fp8_cast_blocks_ex(const void* X, void* Q, float* sfb, int G, int N, int K, int fmt, void* stream);
 
 /* Synchronise `stream`, then read and clear the device status word:
- * FG_OK, or FG_ERR_TIMEOUT if some kernel since the last call gave up a wait. */
+ * FG_OK, or FG_ERR_TIMEOUT if some kernel since the last call gave up a wait, or (debug
+ * build, libfp8gemm_debug.so, compiled with -DFG_DEBUG) FG_ERR_DEVICE_CHECK if a
+ * device-side index check failed.  The first error since the last read wins. */
 fg_status fg_get_device_status(void* stream);
 
 /* Human-readable name of a status code (static storage). */

@@ -27,60 +27,91 @@ if not LIB_PATH.exists():
     raise ImportError(f"{LIB_PATH} is not built; run `python moe_grouped_gemm_08_b200/build.py` "
                       "or __graft_entry__.build()")
 
-_lib = ctypes.CDLL(str(LIB_PATH))
 _vp, _int = ctypes.c_void_p, ctypes.c_int
-_lib.fg_init.argtypes = [_int]
-_lib.fg_init.restype = _int
-_lib.fg_shutdown.argtypes = []
-_lib.fg_shutdown.restype = None
-_lib.fg_m_alignment.restype = _int
-_lib.fg_sfa_ld.argtypes = [_int]
-_lib.fg_sfa_ld.restype = _int
-_lib.fp8_gemm_nt.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
-_lib.fp8_gemm_nt.restype = _int
-_lib.fp8_gemm_grouped_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
-_lib.fp8_gemm_grouped_contiguous.restype = _int
-_lib.fp8_gemm_grouped_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
-_lib.fp8_gemm_grouped_masked.restype = _int
-_lib.fp8_gemm_nt_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
-_lib.fp8_gemm_nt_noalloc.restype = _int
-_lib.fp8_gemm_nt_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp]
-_lib.fp8_gemm_nt_ex.restype = _int
-_lib.fp8_gemm_grouped_contiguous_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
-                                                _vp]
-_lib.fp8_gemm_grouped_contiguous_ex.restype = _int
-_lib.fp8_gemm_grouped_masked_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _vp]
-_lib.fp8_gemm_grouped_masked_ex.restype = _int
-_lib.fp8_cast_rows.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
-_lib.fp8_cast_rows.restype = _int
-_lib.fp8_cast_blocks.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
-_lib.fp8_cast_blocks.restype = _int
-_lib.fp8_cast_rows_ex.argtypes = [_vp, _vp, _vp, _int, _int, _int, _int, _vp]
-_lib.fp8_cast_rows_ex.restype = _int
-_lib.fp8_cast_blocks_ex.argtypes = [_vp, _vp, _vp, _int, _int, _int, _int, _vp]
-_lib.fp8_cast_blocks_ex.restype = _int
-_lib.fg_noalloc_status.argtypes = [_vp]
-_lib.fg_noalloc_status.restype = _int
-_lib.fg_get_device_status.argtypes = [_vp]
-_lib.fg_get_device_status.restype = _int
-_lib.fg_status_string.argtypes = [_int]
-_lib.fg_status_string.restype = ctypes.c_char_p
-_lib.fg_set_dense_path.argtypes = [_int]
-_lib.fg_set_dense_path.restype = _int
-_lib.fg_debug_set_stall.argtypes = [_int]
-_lib.fg_debug_set_stall.restype = _int
-_lib.fg_set_tiled_streamk.argtypes = [_int]
-_lib.fg_set_tiled_streamk.restype = _int
-_lib.fg_set_swap_schedule.argtypes = [_int]
-_lib.fg_set_swap_schedule.restype = _int
-_lib.fg_swap_plan.argtypes = [_int, _int, _int]
-_lib.fg_swap_plan.restype = _int
-_lib.fg_launch_count.argtypes = []
-_lib.fg_launch_count.restype = ctypes.c_uint64
+
+
+def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
+    """Argument and result types of every C ABI entry point (include/fp8gemm.h)."""
+    l.fg_init.argtypes = [_int]
+    l.fg_init.restype = _int
+    l.fg_shutdown.argtypes = []
+    l.fg_shutdown.restype = None
+    l.fg_m_alignment.restype = _int
+    l.fg_sfa_ld.argtypes = [_int]
+    l.fg_sfa_ld.restype = _int
+    l.fp8_gemm_nt.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
+    l.fp8_gemm_nt.restype = _int
+    l.fp8_gemm_grouped_contiguous.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
+    l.fp8_gemm_grouped_contiguous.restype = _int
+    l.fp8_gemm_grouped_masked.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _vp]
+    l.fp8_gemm_grouped_masked.restype = _int
+    l.fp8_gemm_nt_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _vp]
+    l.fp8_gemm_nt_noalloc.restype = _int
+    l.fp8_gemm_nt_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp]
+    l.fp8_gemm_nt_ex.restype = _int
+    l.fp8_gemm_grouped_contiguous_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
+                                                 _vp]
+    l.fp8_gemm_grouped_contiguous_ex.restype = _int
+    l.fp8_gemm_grouped_masked_ex.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int, _vp]
+    l.fp8_gemm_grouped_masked_ex.restype = _int
+    l.fp8_cast_rows.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
+    l.fp8_cast_rows.restype = _int
+    l.fp8_cast_blocks.argtypes = [_vp, _vp, _vp, _int, _int, _int, _vp]
+    l.fp8_cast_blocks.restype = _int
+    l.fp8_cast_rows_ex.argtypes = [_vp, _vp, _vp, _int, _int, _int, _int, _vp]
+    l.fp8_cast_rows_ex.restype = _int
+    l.fp8_cast_blocks_ex.argtypes = [_vp, _vp, _vp, _int, _int, _int, _int, _vp]
+    l.fp8_cast_blocks_ex.restype = _int
+    l.fg_noalloc_status.argtypes = [_vp]
+    l.fg_noalloc_status.restype = _int
+    l.fg_get_device_status.argtypes = [_vp]
+    l.fg_get_device_status.restype = _int
+    l.fg_status_string.argtypes = [_int]
+    l.fg_status_string.restype = ctypes.c_char_p
+    l.fg_set_dense_path.argtypes = [_int]
+    l.fg_set_dense_path.restype = _int
+    l.fg_debug_set_stall.argtypes = [_int]
+    l.fg_debug_set_stall.restype = _int
+    l.fg_set_tiled_streamk.argtypes = [_int]
+    l.fg_set_tiled_streamk.restype = _int
+    l.fg_set_swap_schedule.argtypes = [_int]
+    l.fg_set_swap_schedule.restype = _int
+    l.fg_swap_plan.argtypes = [_int, _int, _int]
+    l.fg_swap_plan.restype = _int
+    l.fg_workspace_bytes.argtypes = []
+    l.fg_workspace_bytes.restype = ctypes.c_size_t
+    l.fp8_gemm_nt_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp, ctypes.c_size_t, _vp]
+    l.fp8_gemm_nt_ws.restype = _int
+    l.fp8_gemm_grouped_contiguous_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
+                                                 _vp, ctypes.c_size_t, _vp]
+    l.fp8_gemm_grouped_contiguous_ws.restype = _int
+    l.fp8_gemm_grouped_masked_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
+                                             _vp, ctypes.c_size_t, _vp]
+    l.fp8_gemm_grouped_masked_ws.restype = _int
+    l.fg_launch_count.argtypes = []
+    l.fg_launch_count.restype = ctypes.c_uint64
+    return l
+
+
+_lib = _declare(ctypes.CDLL(str(LIB_PATH)))
 
 FG_OK = 0
-STATUS_NAMES = {i: _lib.fg_status_string(i).decode() for i in range(7)}
+STATUS_NAMES = {i: _lib.fg_status_string(i).decode() for i in range(8)}
 lib = _lib  # the raw C ABI, for callers that marshal pointers themselves
+DEBUG_LIB_PATH = _HERE / "libfp8gemm_debug.so"
+_debug_lib = None
+
+
+def debug_library() -> ctypes.CDLL:
+    """The debug build of the C ABI (libfp8gemm_debug.so, compiled with -DFG_DEBUG): the same
+    entry points, with device-side index checks that report FG_ERR_DEVICE_CHECK through its own
+    fg_get_device_status.  It keeps its own state (fg_init, workspace, status word)."""
+    global _debug_lib
+    if _debug_lib is None:
+        if not DEBUG_LIB_PATH.exists():
+            raise ImportError(f"{DEBUG_LIB_PATH} is not built; run __graft_entry__.build()")
+        _debug_lib = _declare(ctypes.CDLL(str(DEBUG_LIB_PATH)))
+    return _debug_lib
 
 
 class FP8GemmError(RuntimeError):
@@ -135,6 +166,30 @@ def swap_plan(M: int, N: int, K: int) -> int:
     """Schedule of the small-M kernel for this dense shape: S (2/4/8) cluster split, 1 whole tiles,
     0 stream-K, -1 not applicable."""
     return int(_lib.fg_swap_plan(int(M), int(N), int(K)))
+
+
+def workspace_bytes(device: int | None = None) -> int:
+    """Bytes of a caller-owned split-K workspace for ``device`` (fg_workspace_bytes)."""
+    dev = torch.cuda.current_device() if device is None else int(device)
+    with torch.cuda.device(dev):
+        init(dev)
+        return int(_lib.fg_workspace_bytes())
+
+
+def new_workspace(device=None) -> torch.Tensor:
+    """A zero-filled caller-owned workspace (uint8 CUDA tensor) for the GEMM calls of one stream:
+    calls that may run at the same time need different workspaces."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+    return torch.zeros(workspace_bytes(dev.index), dtype=torch.uint8, device=dev)
+
+
+def _ws(workspace, device):
+    """(pointer, bytes) of a caller-owned workspace, (None, 0) for the library's own."""
+    if workspace is None:
+        return None, 0
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or workspace.device != device:
+        raise ValueError(f"workspace must be a contiguous uint8 tensor on {device}")
+    return workspace.data_ptr(), workspace.numel()
 
 
 def launch_count() -> int:
@@ -212,9 +267,10 @@ def _cdiv(a, b):
     return (a + b - 1) // b
 
 
-def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=None):
+def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=None, workspace=None):
     """Dense C[M,N] = A[M,K] . B[N,K]^T with 1x128 (A) and 128x128 (B) fp32 scales; A and B are
-    e4m3 or e5m2 (from their dtype, or fmt_a / fmt_b for uint8 codes)."""
+    e4m3 or e5m2 (from their dtype, or fmt_a / fmt_b for uint8 codes).  workspace: a caller-owned
+    split-K workspace (new_workspace()), else the library's own."""
     (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb = _f32(sfa, "sfa"), _f32(sfb, "sfb")
     M, K = A.shape
@@ -227,13 +283,14 @@ def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=
     C = _out(C, (M, N), dev)
     with torch.cuda.device(dev):
         init(dev.index)
-        _check(_lib.fp8_gemm_nt_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
-                                   M, N, K, fa, fb, _stream(stream, dev)), "fp8_gemm_nt")
+        wp, wb = _ws(workspace, dev)
+        _check(_lib.fp8_gemm_nt_ws(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
+                                   M, N, K, fa, fb, wp, wb, _stream(stream, dev)), "fp8_gemm_nt")
     return C
 
 
 def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None, stream=None, fmt_a=None,
-                                              fmt_b=None):
+                                              fmt_b=None, workspace=None):
     """M-grouped contiguous: A[M_total,K], B[G,N,K], m_indices[M_total] (-1 = padding)."""
     (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb, m_indices = _f32(sfa, "sfa"), _f32(sfb, "sfb"), _i32(m_indices, "m_indices")
@@ -247,13 +304,15 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None,
     C = _out(C, (M, N), dev)
     with torch.cuda.device(dev):
         init(dev.index)
-        _check(_lib.fp8_gemm_grouped_contiguous_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                                   C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb,
+        wp, wb = _ws(workspace, dev)
+        _check(_lib.fp8_gemm_grouped_contiguous_ws(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                                   C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb, wp, wb,
                                                    _stream(stream, dev)), "fp8_gemm_grouped_contiguous")
     return C
 
 
-def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stream=None, fmt_a=None, fmt_b=None):
+def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stream=None, fmt_a=None, fmt_b=None,
+                                          workspace=None):
     """M-grouped masked: A[G,Mmax,K], masked_m[G] on the device; rows >= masked_m[g] untouched."""
     (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb, masked_m = _f32(sfa, "sfa"), _f32(sfb, "sfb"), _i32(masked_m, "masked_m")
@@ -268,8 +327,9 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stre
     C = _out(C, (G, Mmax, N), dev)
     with torch.cuda.device(dev):
         init(dev.index)
-        _check(_lib.fp8_gemm_grouped_masked_ex(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                               C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb,
+        wp, wb = _ws(workspace, dev)
+        _check(_lib.fp8_gemm_grouped_masked_ws(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
+                                               C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb, wp, wb,
                                                _stream(stream, dev)), "fp8_gemm_grouped_masked")
     return C
 

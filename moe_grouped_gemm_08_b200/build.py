@@ -8,6 +8,7 @@ import subprocess
 HERE = pathlib.Path(__file__).resolve().parent
 ROOT = HERE.parent
 SO = HERE / "libfp8gemm.so"
+SO_DEBUG = HERE / "libfp8gemm_debug.so"  # the same library with the device-side checks (-DFG_DEBUG)
 SOURCES = [HERE / "csrc" / "fp8gemm_api.cu"]
 DEPENDS = SOURCES + [HERE / "csrc" / "fp8_gemm_kernels.cuh", HERE / "csrc" / "fp8_cast_kernels.cuh",
                      HERE / "csrc" / "sm100_ptx.cuh",
@@ -25,20 +26,27 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def build(force: bool = False, verbose: bool = False) -> pathlib.Path:
-    """Compile the library if any source is newer than the built .so."""
-    if not force and SO.exists():
+def _build_one(so: pathlib.Path, extra, force: bool, verbose: bool) -> pathlib.Path:
+    if not force and so.exists():
         newest = max(p.stat().st_mtime for p in DEPENDS)
-        if SO.stat().st_mtime >= newest:
-            return SO
-    tmp = SO.with_suffix(".so.tmp%d" % os.getpid())
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", str(ROOT / "include"), "-I", str(HERE / "csrc"),
+        if so.stat().st_mtime >= newest:
+            return so
+    tmp = so.with_suffix(".so.tmp%d" % os.getpid())
+    cmd = [nvcc(), *NVCC_FLAGS, *extra, "-I", str(ROOT / "include"), "-I", str(HERE / "csrc"),
            *(str(s) for s in SOURCES), "-o", str(tmp)]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
-    os.replace(tmp, SO)
-    return SO
+    os.replace(tmp, so)
+    return so
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> pathlib.Path:
+    """Compile the library (and, with debug=True, its debug build) if any source is newer than
+    the built .so."""
+    if debug:
+        _build_one(SO_DEBUG, ["-DFG_DEBUG"], force, False)
+    return _build_one(SO, [], force, verbose)
 
 
 if __name__ == "__main__":

@@ -48,6 +48,7 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s, far above any legal wait
 constexpr int kErrTimeout = 6;       // FG_ERR_TIMEOUT
+constexpr int kErrDeviceCheck = 7;   // FG_ERR_DEVICE_CHECK (debug builds only)
 constexpr int kMaskedMaxGroups = 1024;
 constexpr int kSwapScaleBytes = 12 * 1024;  // shared memory for staged combined scales (swap kernel)
 constexpr int kSaChunk = 8;                 // K blocks per staged scale chunk (tiled kernel)
@@ -79,6 +80,7 @@ struct TiledParams {
   uint32_t fmt_bits;  // operand formats in instruction-descriptor position (0: both e4m3)
   float* ws;        // stream-K tail: 2 * gridDim.x partial tiles of 128 x BN fp32
   int* counters;    // stream-K tail: one per tile of the last partial wave, zero between launches
+  int counter_cap;  // entries of `counters`
   int sk_overhead;  // < 0: no stream-K tail; else the K blocks a split must save to be taken
 };
 
@@ -88,6 +90,7 @@ struct SwapParams {
   __nv_bfloat16* C;
   float* ws;       // 2 * gridDim.x partial tiles of MP x 128 fp32
   int* counters;   // one per n-tile, zero between launches
+  int counter_cap; // entries of `counters`
   int* status;
   int M, N, K, ld;
   int num_kb;
@@ -105,6 +108,21 @@ __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
 }
 
 __device__ __forceinline__ void report_timeout(int* status) { atomicCAS(status, 0, kErrTimeout); }
+
+// Debug builds (-DFG_DEBUG): device-side checks of indices the kernels derive from their inputs
+// or their schedule -- TMA tile coordinates, expert indices read from m_indices, split-K
+// workspace slots and counters.  A failed check records FG_ERR_DEVICE_CHECK in the status word
+// (first error wins) and the kernel carries on exactly as a release build would; nothing traps.
+#ifdef FG_DEBUG
+#define FG_DCHECK(cond, status)                                           \
+  do {                                                                    \
+    if (!(cond)) atomicCAS((status), 0, ::fg::kErrDeviceCheck);           \
+  } while (0)
+#else
+#define FG_DCHECK(cond, status) \
+  do {                          \
+  } while (0)
+#endif
 
 // Wait for the phase of `bar` with parity `parity` regardless of the abort flag
 // (used only to drain this CTA's own copies after an abort); bounded.
@@ -271,6 +289,7 @@ __device__ __forceinline__ TileInfo tiled_tile(const TiledParams& p, const int* 
     ti.n0 = nb * BN;
     if (MODE == kContiguous) {
       const int g = __ldg(p.m_indices + ti.m0);
+      FG_DCHECK(g >= -1 && g < p.G, p.status);
       ti.live = (g >= 0 && g < p.G);
       ti.g = ti.live ? g : 0;
     } else {
@@ -445,6 +464,8 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         if (!ti.live) continue;
         const int ga = (MODE == kMasked) ? ti.g : 0;
         const int gb = (MODE == kDense) ? 0 : ti.g;
+        FG_DCHECK(ti.m0 >= 0 && ti.m0 < p.M && ti.n0 >= 0 && ti.n0 < p.N && ti.g >= 0 && ti.g < p.G, p.status);
+        FG_DCHECK(it.kb0 >= 0 && it.kb0 < it.kb1 && it.kb1 <= p.num_kb, p.status);
         for (int kb = it.kb0; kb < it.kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           uint8_t* st = smem + stage * STAGE_BYTES;
@@ -593,6 +614,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         const int c_first = sk_owner(tu0, plan.sk_ctas, plan.U);
         const int c_last = sk_owner(tu0 + p.num_kb - 1, plan.sk_ctas, plan.U);
         float4* ws4 = reinterpret_cast<float4*>(p.ws);
+        FG_DCHECK(sk_slot(blockIdx.x, plan.sk_ctas, plan.U, tu0) < 2 * static_cast<int>(gridDim.x) &&
+                      tl >= 0 && tl < p.counter_cap && c_first <= static_cast<int>(blockIdx.x) &&
+                      static_cast<int>(blockIdx.x) <= c_last,
+                  p.status);
         float4* wp = ws4 + static_cast<size_t>(sk_slot(blockIdx.x, plan.sk_ctas, plan.U, tu0)) * TILE_F4 + tid;
 #pragma unroll
         for (int i = 0; i < COLS / 4; ++i)
@@ -640,7 +665,11 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
         cnt = cnt > p.M ? p.M : cnt;
         store_row = m < cnt;
       } else if (MODE == kContiguous) {
-        if (store_row) store_row = __ldg(p.m_indices + m) == ti.g;
+        if (store_row) {
+          const int gi = __ldg(p.m_indices + m);
+          FG_DCHECK(gi >= -1 && gi < p.G, p.status);
+          store_row = gi == ti.g;
+        }
       }
       const int nbase = ti.n0 + h * COLS;
       if (__all_sync(0xffffffffu, store_row)) {
@@ -832,6 +861,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
         const int gb = (MODE == kDense) ? 0 : ti.g;
         const int a_row = ti.m0 + static_cast<int>(rank) * kBlockM;
         const int b_row = ti.n0 + static_cast<int>(rank) * COLS;
+        FG_DCHECK(ti.m0 >= 0 && ti.m0 < p.M && ti.n0 >= 0 && ti.n0 < p.N && ti.g >= 0 && ti.g < p.G, p.status);
         for (int kb = 0; kb < p.num_kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           uint8_t* st = smem + stage * STAGE_BYTES;
@@ -1154,6 +1184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto issue = [&](int u) {
     const int t = u / KB;
     const int kb = u - t * KB;
+    FG_DCHECK(t >= 0 && t < p.n_tiles && t * kBlockM < p.N && kb * kBlockK < p.K, p.status);
     uint8_t* sw = smem + p_stage * STAGE_BYTES;
     mbar_arrive_expect_tx(&full[p_stage], STAGE_BYTES);
     tma_load_2d(sw, &tmW, &full[p_stage], kb * kBlockK, t * kBlockM, pol_w);
@@ -1337,6 +1368,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int c_first = sk_owner(tu0, P, U);
         const int c_last = sk_owner(tu0 + KB - 1, P, U);
         const int slot = 2 * blockIdx.x + (first_segment ? 0 : 1);
+        FG_DCHECK(t < p.counter_cap && c_first <= static_cast<int>(blockIdx.x) &&
+                      static_cast<int>(blockIdx.x) <= c_last && c_first >= 0 && c_last < P,
+                  p.status);
         float* wp = p.ws + static_cast<size_t>(slot) * MP * kBlockM + nl;
 #pragma unroll
         for (int j = 0; j < COLS; ++j) wp[static_cast<size_t>(h * COLS + j) * kBlockM] = acc[j];

@@ -64,6 +64,10 @@ std::atomic<uint64_t> g_launches{0};
 #define FG_TILED_GROUP_MB 48  // L2 budget (MB) for the A rows of one group of m-blocks
 #endif
 constexpr int kTiledBN = FG_TILED_BN;
+#ifndef FG_TILED_BN_MAX
+#define FG_TILED_BN_MAX 256  // widest tile of any tiled-kernel instance (sizes the split-K partials)
+#endif
+static_assert(kTiledBN <= FG_TILED_BN_MAX, "tile wider than the workspace allows");
 constexpr int kTiledStages = FG_TILED_STAGES;
 // CTA-pair kernel: 256 x 192 tiles per pair, each CTA's stage = 128 A rows + 96 B rows
 #ifndef FG_PAIR_BN
@@ -107,6 +111,32 @@ int current_device() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return -1;
   return dev;
+}
+
+// What one GEMM launch uses besides its operands: the SM count, the status word, and the split-K
+// workspace (partial tiles + per-tile counters) -- the library's own (fg_init) or the caller's.
+struct Ctx {
+  int sms = 0;
+  int* status = nullptr;
+  float* ws = nullptr;
+  int* counters = nullptr;
+};
+
+// Split-K workspace layout (library-owned and caller-owned alike): two partial tiles per SM of
+// 128 x max(swap MP, tiled BN) fp32, then kCounterCapacity int counters (zero between launches).
+size_t workspace_partial_bytes(int sms) {
+  return static_cast<size_t>(2) * sms * kBlockM * (kMaxSwapMP > FG_TILED_BN_MAX ? kMaxSwapMP : FG_TILED_BN_MAX) *
+         sizeof(float);
+}
+size_t workspace_bytes_for(int sms) { return workspace_partial_bytes(sms) + kCounterCapacity * sizeof(int); }
+
+Ctx ctx_of(const DeviceState* st) {
+  Ctx c;
+  c.sms = st->sms;
+  c.status = st->status;
+  c.ws = st->ws;
+  c.counters = st->counters;
+  return c;
 }
 
 DeviceState* state_for_current(fg_status* err) {
@@ -220,7 +250,7 @@ fg_status check_common(const void* A, const float* sfa, const void* B, const flo
 }
 
 template <int MODE>
-fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                     const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
                     int fmt_a, int fmt_b) {
   constexpr int BN = kTiledBN;
@@ -262,6 +292,7 @@ fg_status run_tiled(DeviceState* st, const void* A, const float* sfa, const void
 
   p.ws = st->ws;
   p.counters = st->counters;
+  p.counter_cap = kCounterCapacity;
   p.sk_overhead = g_tiled_sk.load(std::memory_order_relaxed);
   // masked: an upper bound (the live tiles are counted on the device)
   const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
@@ -309,7 +340,7 @@ int pair_capacity(int sms, size_t smem) {
 }
 
 template <int MODE>
-fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
   constexpr int BN = kPairBN;
   constexpr int STAGES = kPairStages;
@@ -319,6 +350,7 @@ fg_status run_pair(DeviceState* st, const void* A, const float* sfa, const void*
   p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
   p.ws = nullptr;
   p.counters = nullptr;
+  p.counter_cap = 0;
   p.sk_overhead = -1;
   p.sfa = sfa;
   p.sfb = sfb;
@@ -459,7 +491,7 @@ SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
 }
 
 template <int MP>
-fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+fg_status run_swap(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
   constexpr int STAGES = swap_stages<MP>();
   fg::SwapParams p;
@@ -470,6 +502,7 @@ fg_status run_swap(DeviceState* st, const void* A, const float* sfa, const void*
   p.C = static_cast<__nv_bfloat16*>(C);
   p.ws = st->ws;
   p.counters = st->counters;
+  p.counter_cap = kCounterCapacity;
   p.status = st->status;
   p.M = M;
   p.N = N;
@@ -548,6 +581,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.C = static_cast<__nv_bfloat16*>(C);
   p.ws = reinterpret_cast<float*>(d.base);
   p.counters = reinterpret_cast<int*>(d.base + kNoAllocPartialBytes);
+  p.counter_cap = kNoAllocCounters;
   p.status = p.counters + kNoAllocCounters;
   p.M = M;
   p.N = N;
@@ -603,10 +637,8 @@ fg_status fg_init(int device) {
   if (major != 10 || minor != 0) return FG_ERR_UNSUPPORTED;  // built for sm_100a only
   if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return FG_ERR_CUDA;
   // two partial tiles per CTA: MP x 128 (swap kernel) or 128 x BN (tiled kernel's stream-K tail)
-  const size_t tile_floats = static_cast<size_t>(kBlockM) * (kMaxSwapMP > kTiledBN ? kMaxSwapMP : kTiledBN);
-  const size_t ws_floats = static_cast<size_t>(2) * st.sms * tile_floats;
   if (cudaMalloc(&st.status, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
-  if (cudaMalloc(&st.ws, ws_floats * sizeof(float)) != cudaSuccess) return FG_ERR_CUDA;
+  if (cudaMalloc(&st.ws, workspace_partial_bytes(st.sms)) != cudaSuccess) return FG_ERR_CUDA;
   if (cudaMalloc(&st.counters, kCounterCapacity * sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
   if (cudaMemset(st.status, 0, sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
   if (cudaMemset(st.counters, 0, kCounterCapacity * sizeof(int)) != cudaSuccess) return FG_ERR_CUDA;
@@ -668,16 +700,39 @@ static bool valid_formats(int fmt_a, int fmt_b) {
   return (fmt_a == FG_E4M3 || fmt_a == FG_E5M2) && (fmt_b == FG_E4M3 || fmt_b == FG_E5M2);
 }
 
-fg_status fp8_gemm_nt_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
-                         int K, int fmt_a, int fmt_b, void* stream) {
+size_t fg_workspace_bytes(void) {
+  fg_status s;
+  const DeviceState* st = state_for_current(&s);
+  return st ? workspace_bytes_for(st->sms) : 0;
+}
+
+// Launch context of a call: the library's workspace (workspace == NULL, workspace_bytes == 0) or
+// the caller's (at least fg_workspace_bytes(), 16-byte aligned).
+static fg_status resolve_ctx(void* workspace, size_t workspace_bytes, Ctx* out) {
+  fg_status s;
+  const DeviceState* st = state_for_current(&s);
+  if (!st) return s;
+  *out = ctx_of(st);
+  if (workspace == nullptr) return workspace_bytes == 0 ? FG_OK : FG_ERR_INVALID_ARG;
+  if (!aligned(workspace, 16)) return FG_ERR_ALIGNMENT;
+  if (workspace_bytes < workspace_bytes_for(st->sms)) return FG_ERR_INVALID_ARG;
+  out->ws = static_cast<float*>(workspace);
+  out->counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + workspace_partial_bytes(st->sms));
+  return FG_OK;
+}
+
+fg_status fp8_gemm_nt_ws(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
+                         int K, int fmt_a, int fmt_b, void* workspace, size_t workspace_bytes, void* stream) {
   if (M < 0 || N < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return FG_OK;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
   if (s != FG_OK) return s;
   if (static_cast<long long>(M) * K >= (1ll << 40) || static_cast<long long>(N) * K >= (1ll << 40))
     return FG_ERR_UNSUPPORTED;
-  DeviceState* st = state_for_current(&s);
-  if (!st) return s;
+  Ctx ctx;
+  s = resolve_ctx(workspace, workspace_bytes, &ctx);
+  if (s != FG_OK) return s;
+  const Ctx* st = &ctx;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const int path = g_dense_path.load();
   const bool swap = (path == 2) || (path == 0 && M <= kMaxSwapMP);
@@ -691,14 +746,19 @@ fg_status fp8_gemm_nt_ex(const void* A, const float* sfa, const void* B, const f
   return run_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
 }
 
+fg_status fp8_gemm_nt_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
+                         int K, int fmt_a, int fmt_b, void* stream) {
+  return fp8_gemm_nt_ws(A, sfa, B, sfb, C, M, N, K, fmt_a, fmt_b, nullptr, 0, stream);
+}
+
 fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
                       int K, void* stream) {
   return fp8_gemm_nt_ex(A, sfa, B, sfb, C, M, N, K, FG_E4M3, FG_E4M3, stream);
 }
 
-fg_status fp8_gemm_grouped_contiguous_ex(const void* A, const float* sfa, const void* B, const float* sfb,
+fg_status fp8_gemm_grouped_contiguous_ws(const void* A, const float* sfa, const void* B, const float* sfb,
                                          void* C, const int* m_indices, int M_total, int G, int N, int K, int fmt_a,
-                                         int fmt_b, void* stream) {
+                                         int fmt_b, void* workspace, size_t workspace_bytes, void* stream) {
   if (M_total < 0 || N < 0 || G < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
   if (M_total == 0 || N == 0) return FG_OK;
   if (G == 0) return FG_ERR_INVALID_ARG;
@@ -708,10 +768,18 @@ fg_status fp8_gemm_grouped_contiguous_ex(const void* A, const float* sfa, const 
   if (!aligned(m_indices, 4)) return FG_ERR_ALIGNMENT;
   if (static_cast<long long>(M_total) * K >= (1ll << 40) || static_cast<long long>(G) * N * K >= (1ll << 40))
     return FG_ERR_UNSUPPORTED;
-  DeviceState* st = state_for_current(&s);
-  if (!st) return s;
-  return run_tiled<fg::kContiguous>(st, A, sfa, B, sfb, C, m_indices, nullptr, M_total, G, N, K,
+  Ctx ctx;
+  s = resolve_ctx(workspace, workspace_bytes, &ctx);
+  if (s != FG_OK) return s;
+  return run_tiled<fg::kContiguous>(&ctx, A, sfa, B, sfb, C, m_indices, nullptr, M_total, G, N, K,
                                     static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
+}
+
+fg_status fp8_gemm_grouped_contiguous_ex(const void* A, const float* sfa, const void* B, const float* sfb,
+                                         void* C, const int* m_indices, int M_total, int G, int N, int K, int fmt_a,
+                                         int fmt_b, void* stream) {
+  return fp8_gemm_grouped_contiguous_ws(A, sfa, B, sfb, C, m_indices, M_total, G, N, K, fmt_a, fmt_b, nullptr, 0,
+                                        stream);
 }
 
 fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
@@ -719,9 +787,9 @@ fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const voi
   return fp8_gemm_grouped_contiguous_ex(A, sfa, B, sfb, C, m_indices, M_total, G, N, K, FG_E4M3, FG_E4M3, stream);
 }
 
-fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+fg_status fp8_gemm_grouped_masked_ws(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                                      const int* masked_m, int G, int Mmax, int N, int K, int fmt_a, int fmt_b,
-                                     void* stream) {
+                                     void* workspace, size_t workspace_bytes, void* stream) {
   if (G < 0 || Mmax < 0 || N < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
   if (G == 0 || Mmax == 0 || N == 0) return FG_OK;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
@@ -731,13 +799,20 @@ fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void
   if (G > fg::kMaskedMaxGroups) return FG_ERR_UNSUPPORTED;
   if (static_cast<long long>(G) * Mmax * K >= (1ll << 40) || static_cast<long long>(G) * N * K >= (1ll << 40))
     return FG_ERR_UNSUPPORTED;
-  DeviceState* st = state_for_current(&s);
-  if (!st) return s;
+  Ctx ctx;
+  s = resolve_ctx(workspace, workspace_bytes, &ctx);
+  if (s != FG_OK) return s;
   if (g_dense_path.load() == 3)
-    return run_pair<fg::kMasked>(st, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K, static_cast<cudaStream_t>(stream),
+    return run_pair<fg::kMasked>(&ctx, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K, static_cast<cudaStream_t>(stream),
                                  fmt_a, fmt_b);
-  return run_tiled<fg::kMasked>(st, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
+  return run_tiled<fg::kMasked>(&ctx, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
                                 static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
+}
+
+fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                                     const int* masked_m, int G, int Mmax, int N, int K, int fmt_a, int fmt_b,
+                                     void* stream) {
+  return fp8_gemm_grouped_masked_ws(A, sfa, B, sfb, C, masked_m, G, Mmax, N, K, fmt_a, fmt_b, nullptr, 0, stream);
 }
 
 fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
@@ -862,6 +937,7 @@ const char* fg_status_string(fg_status status) {
     case FG_ERR_NOT_INITIALIZED: return "FG_ERR_NOT_INITIALIZED";
     case FG_ERR_CUDA: return "FG_ERR_CUDA";
     case FG_ERR_TIMEOUT: return "FG_ERR_TIMEOUT";
+    case FG_ERR_DEVICE_CHECK: return "FG_ERR_DEVICE_CHECK";
   }
   return "FG_ERR_UNKNOWN";
 }

@@ -114,3 +114,26 @@ def test_cast_argument_errors():
         assert f(P16, P16, P16, 0, 4, 128, NULL) == 0            # G = 0: no-op, nothing launched
         assert f(P16, P16, P16, 1, 0, 128, NULL) == 0            # no rows: no-op
     assert cast_blocks(P16, P16, P16, 70000, 4, 128, NULL) == 3  # more groups than a grid axis holds
+
+
+def test_debug_build_exports_the_same_symbols():
+    lib = fg.debug_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} missing from the debug build"
+    assert fg.STATUS_NAMES[7] == "FG_ERR_DEVICE_CHECK"
+    assert lib.fg_status_string(7) == b"FG_ERR_DEVICE_CHECK"
+
+
+def test_workspace_entry_points_check_arguments_first():
+    L = fg.lib
+    if not torch.cuda.is_available():
+        assert L.fg_workspace_bytes() == 0  # no fg_init on this device
+        # arguments valid, no device state: not initialised, nothing launched
+        assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 0, 0, P16, 1 << 30, NULL) == 4
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 120, 0, 0, P16, 1 << 30, NULL) == 2   # K % 16
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 2, 0, P16, 1 << 30, NULL) == 1   # format
+    assert L.fp8_gemm_grouped_contiguous_ws(P16, P16, P16, P16, P16, NULL, 256, 2, 128, 128, 0, 0, P16, 1 << 30,
+                                            NULL) == 1
+    assert L.fp8_gemm_grouped_masked_ws(P16, P16, P16, P16, P16, P16, 2000, 64, 128, 128, 0, 0, P16, 1 << 30,
+                                        NULL) == 3
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 0, 128, 128, 0, 0, NULL, 0, NULL) == 0  # M = 0: no-op
