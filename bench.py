@@ -197,14 +197,14 @@ def upload(case, dev):
     return d
 
 
-def call(fg, case, d, stream=None):
+def call(fg, case, d, stream=None, static_b=False):
     if case["kind"] == "masked":
         return fg.m_grouped_gemm_fp8_fp8_bf16_nt_masked(d["A"], d["sfa"], d["B"], d["sfb"], d["masked_m"],
                                                         C=d["C"], stream=stream)
     if case["kind"] == "contiguous":
         return fg.m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(d["A"], d["sfa"], d["B"], d["sfb"], d["m_indices"],
                                                             C=d["C"], stream=stream)
-    return fg.gemm_fp8_fp8_bf16_nt(d["A"], d["sfa"], d["B"], d["sfb"], C=d["C"], stream=stream)
+    return fg.gemm_fp8_fp8_bf16_nt(d["A"], d["sfa"], d["B"], d["sfb"], C=d["C"], stream=stream, static_b=static_b)
 
 
 _CUDART = None
@@ -450,7 +450,7 @@ def run_cast(args, rank, world, local):
 
 
 # ---------------------------------------------------------------------------- our arm
-def measure_workload(fg, name, wl, args, dev, stream, world, local):
+def measure_workload(fg, name, wl, args, dev, stream, world, local, static_b=False):
     """Time one workload: each step (one call per GEMM of the workload) is replayed from a CUDA
     graph, inputs rotating over enough copies that every launch reads HBM.  Returns the workload's
     result dict, its cases and the device copies (for the end-to-end leg)."""
@@ -467,7 +467,7 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local):
     # eager warm-up call per case (sets kernel attributes before capture), then capture one graph per copy
     with torch.cuda.stream(stream):
         for c, d in zip(cases, devs[0]):
-            call(fg, c, d, stream=stream)
+            call(fg, c, d, stream=stream, static_b=static_b)
     stream.synchronize()
     launches_before = fg.launch_count()
     graphs = []       # kernels only: the timed region (consecutive launches may overlap via PDL)
@@ -475,7 +475,7 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
             for c, d in zip(cases, devs[r]):
-                call(fg, c, d, stream=stream)
+                call(fg, c, d, stream=stream, static_b=static_b)
         graphs.append(g)
     launches_per_step = (fg.launch_count() - launches_before) // rot
     egraphs, gevents = [], []  # the same step with an event node around every launch: per-shape times
@@ -488,7 +488,7 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local):
         with torch.cuda.graph(g, stream=stream):
             for i, (c, d) in enumerate(zip(cases, devs[r])):
                 record_event_node(evs[i], stream)
-                call(fg, c, d, stream=stream)
+                call(fg, c, d, stream=stream, static_b=static_b)
             record_event_node(evs[-1], stream)
         egraphs.append(g)
         gevents.append(evs)
@@ -583,7 +583,8 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local):
            "hbm_gbs": round(step_bytes * args.steps * world / (elapsed_ms * 1e-3) / 1e9, 1),
            "config": {"workload": name, "shapes": [w["name"] for w in wl],
                       "l2": f"inputs rotate over {rot} copies ({rot * step_in_bytes / 1e6:.0f} MB > L2)",
-                      "graph": "each step replayed from a CUDA graph"},
+                      "graph": "each step replayed from a CUDA graph",
+                      "static_b": static_b},
            "shapes": shapes, "shapes_timing": "event node around each launch, separate pass after the timed region",
            "roofline": roof, "gpu_launches": launches_per_step * args.steps,
            "clocks": clocks.summary(t_wall0, t_wall1), "device_status": fg.STATUS_NAMES.get(status, status)}
@@ -605,7 +606,11 @@ def run_ours(args, rank, world, local):
         fg.set_swap_schedule(args.swap_schedule)
     stream = torch.cuda.Stream(device=dev)
     name, wl = workload_list(args.workload, args.shape)
-    res, cases, devs, step_flops = measure_workload(fg, name, wl, args, dev, stream, world, local)
+    # The weights of a decode step are loaded once and never rewritten, so the dense calls declare
+    # them static (FG_FLAG_STATIC_B: weight tiles may load before the preceding launch ends);
+    # --no-static-b times the fully stream-ordered form, which is also reported under "workloads".
+    res, cases, devs, step_flops = measure_workload(fg, name, wl, args, dev, stream, world, local,
+                                                    static_b=args.static_b)
 
     # end to end through the public API with host buffers: H2D of the step's inputs, GEMMs, D2H of C
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -625,7 +630,7 @@ def run_ours(args, rank, world, local):
         for c, h, d, o in zip(cases, host, devs[0], outs):
             for key, t in h.items():
                 d[key].copy_(t, non_blocking=True)
-            call(fg, c, d, stream=stream)
+            call(fg, c, d, stream=stream)  # B is copied in just before: not static here
             o.copy_(d["C"], non_blocking=True)
 
     with torch.cuda.stream(stream):
@@ -666,14 +671,18 @@ def run_ours(args, rank, world, local):
 
     # the other configurations, timed the same way in the same process (same steps and warm-up)
     extra = [x for x in (args.also.split(",") if args.also else []) if x and x != name]
+    if args.static_b and not args.shape and any(c["kind"] == "dense" for c in cases):
+        extra = [name + ":ordered"] + extra
     if extra and not args.shape:
         line["workloads"] = {}
         for other in extra:
-            oname, owl = workload_list(other)
-            ores, ocases, odevs, _ = measure_workload(fg, oname, owl, args, dev, stream, world, local)
+            base, _, mode = other.partition(":")
+            oname, owl = workload_list(base)
+            ores, ocases, odevs, _ = measure_workload(fg, oname, owl, args, dev, stream, world, local,
+                                                      static_b=args.static_b and mode != "ordered")
             del ocases, odevs
             torch.cuda.empty_cache()
-            line["workloads"][oname] = ores
+            line["workloads"][oname + (" (stream-ordered weights)" if mode == "ordered" else "")] = ores
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -691,6 +700,8 @@ def main():
                     help="comma-separated workloads timed after the headline one in the same run, reported "
                          "under the 'workloads' key (empty: none)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-static-b", dest="static_b", action="store_false",
+                    help="do not declare the weights static (FG_FLAG_STATIC_B) in the timed dense calls")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],

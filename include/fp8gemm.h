@@ -140,6 +140,17 @@ fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void
  * 0 if fg_init was not called for the device. */
 size_t fg_workspace_bytes(void);
 
+/* Call options (the `flags` argument of the _ws entry points), or-ed together.
+ * FG_FLAG_STATIC_B: B and sfb are not written by the kernel that immediately precedes this
+ *   call on its stream (weights loaded once and reused, as in inference).  The kernel may
+ *   then start loading weight tiles before that kernel has finished (it still waits for it
+ *   before touching A, sfa, C or the workspace), which hides the hand-over between
+ *   back-to-back launches.  Taken by the small-M kernel (dense M <= 128); the other kernels
+ *   ignore it.  Results are identical with and without it; a caller that breaks the
+ *   promise (e.g. casts B with fp8_cast_blocks right before the call) may get results
+ *   computed from stale weights. */
+#define FG_FLAG_STATIC_B 1u
+
 /* The three GEMMs with a caller-owned workspace (device memory, 16-byte aligned, at least
  * fg_workspace_bytes() bytes, zero-filled once before its first use, e.g. with
  * cudaMemsetAsync).  Every kernel leaves the counters at zero again when it finishes, so
@@ -148,18 +159,19 @@ size_t fg_workspace_bytes(void);
  * with FG_ERR_TIMEOUT (fg_get_device_status) the caller zero-fills its workspace again.
  * workspace == NULL with workspace_bytes == 0 uses the library's own workspace (the _ex
  * entry points); a workspace that is too small is FG_ERR_INVALID_ARG, a misaligned one
- * FG_ERR_ALIGNMENT.  Everything else is as for the _ex entry points. */
+ * FG_ERR_ALIGNMENT.  flags: FG_FLAG_* options (0 for none; an unknown bit is
+ * FG_ERR_INVALID_ARG).  Everything else is as for the _ex entry points. */
 fg_status fp8_gemm_nt_ws(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                         int M, int N, int K, int fmt_a, int fmt_b, void* workspace,
+                         int M, int N, int K, int fmt_a, int fmt_b, unsigned flags, void* workspace,
                          size_t workspace_bytes, void* stream);
 fg_status fp8_gemm_grouped_contiguous_ws(const void* A, const float* sfa, const void* B, const float* sfb,
                                          void* C, const int* m_indices, int M_total, int G, int N, int K,
-                                         int fmt_a, int fmt_b, void* workspace, size_t workspace_bytes,
-                                         void* stream);
+                                         int fmt_a, int fmt_b, unsigned flags, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 fg_status fp8_gemm_grouped_masked_ws(const void* A, const float* sfa, const void* B, const float* sfb,
                                      void* C, const int* masked_m, int G, int Mmax, int N, int K,
-                                     int fmt_a, int fmt_b, void* workspace, size_t workspace_bytes,
-                                     void* stream);
+                                     int fmt_a, int fmt_b, unsigned flags, void* workspace,
+                                     size_t workspace_bytes, void* stream);
 
 /* Allocation-free variant of fp8_gemm_nt, for callers that cannot allocate device
  * memory: code running inside another framework's memory pool or a pre-planned
@@ -235,6 +247,13 @@ const char* fg_status_string(fg_status status);
  * always takes the one-CTA tiled kernel.  Returns the previous value; an unknown
  * value is ignored. */
 int fg_set_dense_path(int path);
+
+/* Output tile width (columns of N per tile) of the tiled and CTA-pair kernels, process-wide:
+ * 0 (default) = automatic, or 128, 192 or 256 to force a width (the CTA-pair kernel has
+ * 192 and 256; it takes 192 for a forced 128).  Widths other than these are ignored.
+ * Results are identical in every width up to fp32 summation order of split tiles.
+ * Returns the previous value. */
+int fg_set_tile_n(int bn);
 
 /* Stream-K tail of the tiled kernel (dense M > 128, contiguous, masked), process-wide.
  * The tiles are walked whole in waves over the SMs; when the last wave is partial

@@ -72,6 +72,8 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_set_dense_path.restype = _int
     l.fg_debug_set_stall.argtypes = [_int]
     l.fg_debug_set_stall.restype = _int
+    l.fg_set_tile_n.argtypes = [_int]
+    l.fg_set_tile_n.restype = _int
     l.fg_set_tiled_streamk.argtypes = [_int]
     l.fg_set_tiled_streamk.restype = _int
     l.fg_set_swap_schedule.argtypes = [_int]
@@ -80,13 +82,14 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_swap_plan.restype = _int
     l.fg_workspace_bytes.argtypes = []
     l.fg_workspace_bytes.restype = ctypes.c_size_t
-    l.fp8_gemm_nt_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _vp, ctypes.c_size_t, _vp]
+    l.fp8_gemm_nt_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, ctypes.c_uint, _vp,
+                                 ctypes.c_size_t, _vp]
     l.fp8_gemm_nt_ws.restype = _int
     l.fp8_gemm_grouped_contiguous_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
-                                                 _vp, ctypes.c_size_t, _vp]
+                                                 ctypes.c_uint, _vp, ctypes.c_size_t, _vp]
     l.fp8_gemm_grouped_contiguous_ws.restype = _int
     l.fp8_gemm_grouped_masked_ws.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _int, _int, _int, _int,
-                                             _vp, ctypes.c_size_t, _vp]
+                                             ctypes.c_uint, _vp, ctypes.c_size_t, _vp]
     l.fp8_gemm_grouped_masked_ws.restype = _int
     l.fg_launch_count.argtypes = []
     l.fg_launch_count.restype = ctypes.c_uint64
@@ -147,6 +150,12 @@ def set_dense_path(path: int) -> int:
     """0 automatic, 1 one-CTA tiled kernel (dense), 2 swap-AB stream-K (dense, M <= 128),
     3 CTA-pair kernel (dense and masked). Returns the old value."""
     return int(_lib.fg_set_dense_path(int(path)))
+
+
+def set_tile_n(bn: int) -> int:
+    """Output tile width of the tiled / CTA-pair kernels: 0 automatic, or 128, 192, 256. Returns the
+    old value."""
+    return int(_lib.fg_set_tile_n(int(bn)))
 
 
 def set_tiled_streamk(overhead: int) -> int:
@@ -267,10 +276,16 @@ def _cdiv(a, b):
     return (a + b - 1) // b
 
 
-def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=None, workspace=None):
+FLAG_STATIC_B = 1  # FG_FLAG_STATIC_B
+
+
+def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=None, workspace=None,
+                         static_b=False):
     """Dense C[M,N] = A[M,K] . B[N,K]^T with 1x128 (A) and 128x128 (B) fp32 scales; A and B are
     e4m3 or e5m2 (from their dtype, or fmt_a / fmt_b for uint8 codes).  workspace: a caller-owned
-    split-K workspace (new_workspace()), else the library's own."""
+    split-K workspace (new_workspace()), else the library's own.  static_b: the caller promises that
+    B and sfb are not written by the kernel launched just before on the stream (FG_FLAG_STATIC_B),
+    so weight loading may start before that kernel ends."""
     (A, fa), (B, fb) = _bytes(A, "A", fmt_a), _bytes(B, "B", fmt_b)
     sfa, sfb = _f32(sfa, "sfa"), _f32(sfb, "sfb")
     M, K = A.shape
@@ -285,7 +300,8 @@ def gemm_fp8_fp8_bf16_nt(A, sfa, B, sfb, C=None, stream=None, fmt_a=None, fmt_b=
         init(dev.index)
         wp, wb = _ws(workspace, dev)
         _check(_lib.fp8_gemm_nt_ws(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(), C.data_ptr(),
-                                   M, N, K, fa, fb, wp, wb, _stream(stream, dev)), "fp8_gemm_nt")
+                                   M, N, K, fa, fb, FLAG_STATIC_B if static_b else 0, wp, wb,
+                                   _stream(stream, dev)), "fp8_gemm_nt")
     return C
 
 
@@ -306,7 +322,7 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_contiguous(A, sfa, B, sfb, m_indices, C=None,
         init(dev.index)
         wp, wb = _ws(workspace, dev)
         _check(_lib.fp8_gemm_grouped_contiguous_ws(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                                   C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb, wp, wb,
+                                                   C.data_ptr(), m_indices.data_ptr(), M, G, N, K, fa, fb, 0, wp, wb,
                                                    _stream(stream, dev)), "fp8_gemm_grouped_contiguous")
     return C
 
@@ -329,7 +345,7 @@ def m_grouped_gemm_fp8_fp8_bf16_nt_masked(A, sfa, B, sfb, masked_m, C=None, stre
         init(dev.index)
         wp, wb = _ws(workspace, dev)
         _check(_lib.fp8_gemm_grouped_masked_ws(A.data_ptr(), sfa.data_ptr(), B.data_ptr(), sfb.data_ptr(),
-                                               C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb, wp, wb,
+                                               C.data_ptr(), masked_m.data_ptr(), G, Mmax, N, K, fa, fb, 0, wp, wb,
                                                _stream(stream, dev)), "fp8_gemm_grouped_masked")
     return C
 

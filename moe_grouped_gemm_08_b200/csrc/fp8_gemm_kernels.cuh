@@ -54,9 +54,15 @@ constexpr int kSwapScaleBytes = 12 * 1024;  // shared memory for staged combined
 constexpr int kSaChunk = 8;                 // K blocks per staged scale chunk (tiled kernel)
 constexpr int kTiledThreads = 384;          // tiled kernel: three warpgroups
 constexpr int kTiledLaunchRegs = 168;       // registers per thread the tiled kernel is launched with
-constexpr int kPromoRegs = 232;             // after setmaxnreg: promotion warpgroups ...
-constexpr int kCtrlRegs = 40;               // ... and the producer / MMA warpgroup
-static_assert(2 * 128 * kPromoRegs + 128 * kCtrlRegs <= kTiledThreads * kTiledLaunchRegs, "register split");
+// Registers per thread after setmaxnreg, by tile width: the two promotion warpgroups hold the
+// fp32 accumulators and a TMEM slice; the producer / MMA warpgroup needs more with the deeper ring
+// and four TMEM buffers of the 128-wide tile.  Both must add up to at most the launch budget.
+template <int BN>
+struct RegSplit {
+  static constexpr int promo = BN == 128 ? 216 : 232;
+  static constexpr int ctrl = BN == 128 ? 72 : 40;
+  static_assert(2 * 128 * promo + 128 * ctrl <= kTiledThreads * kTiledLaunchRegs, "register split");
+};
 
 enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
@@ -100,6 +106,8 @@ struct SwapParams {
   int tile_aligned;   // 1: CTA c takes whole tiles [c*T/P, (c+1)*T/P) (no split tiles, no fix-up)
   int cluster;        // S > 1: the S CTAs of cluster t split tile t in K and sum it through
                       // distributed shared memory (launched with cluster dims S, grid = tiles * S)
+  int static_b;       // 1: B and sfb are not written by the preceding kernel of the stream, so the
+                      // weight tiles of the first ring stages are loaded before waiting for it
 };
 
 __device__ __forceinline__ uint8_t* align_1024(uint8_t* p) {
@@ -344,6 +352,68 @@ __device__ __forceinline__ void store_scale_chunk(float* buf, int tid, const Sca
   if (tid < 2 * kSaChunk) buf[kSaChunk * kBlockM + tid] = r.b;
 }
 
+// One K block of promotion for one thread: the thread's 32 * NCH columns of the TMEM partial at
+// taddr (its lane, consecutive columns) are read and added, times the block's scale -- s0, or s1
+// for the 32-column chunks whose bit is set in hi_mask (the second 128-column sfb block) -- into
+// the accumulator pairs acc[0 .. 16 NCH) with the packed FMA.  `release` (executed by the whole
+// warp) hands the TMEM buffer back as soon as every chunk has landed in registers.
+// PIPE = false: every chunk is loaded, one wait, then all are added (one load round trip per K
+//   block; 32 NCH registers of slice).
+// PIPE = true: two chunks in flight at a time, chunk i+1 loading while chunk i is added (64
+//   registers of slice, so 128 x 256 tiles fit the register budget).
+template <int NCH, int PIPE, typename Release>
+__device__ __forceinline__ void promote_kblock(uint32_t taddr, float2* acc, float s0, float s1, uint32_t hi_mask,
+                                               Release&& release) {
+  // add W columns (W/2 pairs) of chunk c (c in units of W columns) to the accumulators
+  auto add = [&](const uint32_t* v, int c, int W) {
+    const int i = c * W / 32;  // 32-column chunk: which sfb block
+    const float sc = ((hi_mask >> i) & 1u) ? s1 : s0;
+    const float2 s2 = make_float2(sc, sc);
+#pragma unroll
+    for (int j = 0; j < W / 2; ++j)
+      acc[c * W / 2 + j] = __ffma2_rn(make_float2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])), s2,
+                                      acc[c * W / 2 + j]);
+  };
+  if constexpr (PIPE == 0) {
+    uint32_t v[NCH][32];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) tmem_ld_32x32b_x32(taddr + 32 * i, v[i]);
+    tmem_wait_ld();
+    release();
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) add(v[i], i, 32);
+  } else if constexpr (PIPE == 1) {
+    uint32_t va[32], vb[32];
+    tmem_ld_32x32b_x32(taddr, va);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      if (i + 1 < NCH) {
+        tmem_ld_32x32b_x32(taddr + 32 * (i + 1), (i & 1) ? va : vb);
+      } else {
+        release();
+      }
+      add((i & 1) ? vb : va, i, 32);
+      if (i + 1 < NCH) tmem_wait_ld();
+    }
+  } else {
+    constexpr int N16 = 2 * NCH;
+    uint32_t va[16], vb[16];
+    tmem_ld_32x32b_x16(taddr, va);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < N16; ++i) {
+      if (i + 1 < N16) {
+        tmem_ld_32x32b_x16(taddr + 16 * (i + 1), (i & 1) ? va : vb);
+      } else {
+        release();
+      }
+      add((i & 1) ? vb : va, i, 16);
+      if (i + 1 < N16) tmem_wait_ld();
+    }
+  }
+}
+
 // Output staging of one promotion warp: its 32 rows x COLS columns as COLS/32 boxes of 32 x 32
 // bf16 (64-byte rows, 64-byte swizzle: the 16-byte chunk c of row r sits at chunk c ^ ((r/2)%4)),
 // the layout the C tensor map stores from.
@@ -351,15 +421,15 @@ constexpr int kStoreBoxBytes = 32 * 64;
 
 // Kernel 1 warp roles (384 threads, three warpgroups):
 //   warpgroup 0 (warps 0-3) and 1 (warps 4-7): promotion + epilogue, column halves 0 and 1; each
-//     raises its register budget to kPromoRegs so a thread can hold the BN/2 fp32 accumulators of
+//     raises its register budget (RegSplit) so a thread can hold the BN/2 fp32 accumulators of
 //     its row and one whole BN/2-column slice loaded from TMEM;
 //   warpgroup 2: warp 8 TMA producer, warp 9 TMEM owner + MMA issuer, warps 10-11 idle; it lowers
-//     its budget to kCtrlRegs.  The split assumes the kernel is launched with kTiledLaunchRegs
+//     its budget.  The split assumes the kernel is launched with kTiledLaunchRegs
 //     registers per thread, which the host checks before every launch.
 // BN = 192 keeps one slice read (three 32-column TMEM loads) per K block within the register
 // budget, so each TMEM buffer is handed back after a single load round trip; two buffers of 192
 // columns fit the 512 TMEM columns.
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? 2 : 0)>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
@@ -452,7 +522,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 
   if (warp >= kPromoWarps) {
     // ================================================ warpgroup 2: producer, MMA, idle warps
-    reg_dealloc<kCtrlRegs>();
+    reg_dealloc<RegSplit<BN>::ctrl>();
     if (warp == kProducerWarp && lane == 0) {
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0;
@@ -509,7 +579,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
     }
   } else {
     // ================================================ warpgroups 0-1: promotion + epilogue
-    reg_alloc<kPromoRegs>();
+    reg_alloc<RegSplit<BN>::promo>();
     const int q = warp & 3;
     const int h = warp >> 2;
     const int row = q * 32 + lane;
@@ -575,23 +645,12 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
           if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
-          uint32_t v[NCH][32];
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) tmem_ld_32x32b_x32(taddr + 32 * i, v[i]);
-          tmem_wait_ld();
           // whole slice read: hand the TMEM buffer back to the MMA
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[tb]);
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const float s = ((hi_mask >> i) & 1u) ? s1 : s0;
-            const float2 s2 = make_float2(s, s);
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              acc[16 * i + j] = __ffma2_rn(make_float2(__uint_as_float(v[i][2 * j]), __uint_as_float(v[i][2 * j + 1])),
-                                           s2, acc[16 * i + j]);
-          }
+          promote_kblock<NCH, PIPE>(taddr, acc, s0, s1, hi_mask, [&]() {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[tb]);
+          });
           if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }
         if (!ok) break;
@@ -752,7 +811,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 // tempty[b] of the leader counts the promotion warps of both CTAs.  Cluster barriers only right
 // after set-up and right before teardown, which every thread of both CTAs reaches; every other
 // wait is bounded.
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? 2 : 0)>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
@@ -847,7 +906,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
 
   if (warp >= kPromoWarps) {
     // ================================================ warpgroup 2: producer, MMA, idle warps
-    reg_dealloc<kCtrlRegs>();
+    reg_dealloc<RegSplit<BN>::ctrl>();
     if (warp == kProducerWarp && lane == 0) {
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0;
@@ -911,7 +970,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     }
   } else {
     // ================================================ warpgroups 0-1: promotion + epilogue
-    reg_alloc<kPromoRegs>();
+    reg_alloc<RegSplit<BN>::promo>();
     const int q = warp & 3;
     const int h = warp >> 2;
     const int row = q * 32 + lane;
@@ -970,22 +1029,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
           if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t taddr = tmem_base + lane_off + tb * BN + h * COLS;
-          uint32_t v[NCH][32];
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) tmem_ld_32x32b_x32(taddr + 32 * i, v[i]);
-          tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(tempty_leader + tb * 8);
-#pragma unroll
-          for (int i = 0; i < NCH; ++i) {
-            const float s = ((hi_mask >> i) & 1u) ? s1 : s0;
-            const float2 s2 = make_float2(s, s);
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              acc[16 * i + j] = __ffma2_rn(make_float2(__uint_as_float(v[i][2 * j]), __uint_as_float(v[i][2 * j + 1])),
-                                           s2, acc[16 * i + j]);
-          }
+          promote_kblock<NCH, PIPE>(taddr, acc, s0, s1, hi_mask, [&]() {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_leader + tb * 8);
+          });
           if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }
         if (!ok) break;
@@ -1208,13 +1256,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // Everything above overlaps the previous kernel's tail; from here on global memory is touched.
+  // Weights that the preceding kernel does not write (static_b) start streaming before the wait
+  // for it: the weight half of each of the first ring stages (the token half, which that kernel
+  // may produce, follows the wait).  Each stage's barrier is armed for the whole stage at once.
+  int pre = 0;
+  if (p.static_b && warp == kProducerWarp && lane == 0) {
+    pre = (u_end - u_begin) < STAGES ? (u_end - u_begin) : STAGES;
+    for (int s = 0; s < pre; ++s) {
+      const int u = u_begin + s;
+      const int t = u / KB;
+      const int kb = u - t * KB;
+      FG_DCHECK(t >= 0 && t < p.n_tiles && t * kBlockM < p.N && kb * kBlockK < p.K, p.status);
+      mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+      tma_load_2d(smem + s * STAGE_BYTES, &tmW, &full[s], kb * kBlockK, t * kBlockM, pol_w);
+    }
+  }
+  // Everything above overlaps the previous kernel's tail; from here on global memory is touched
+  // (apart from the weight loads above).
   pdl_wait_prior_grid();
   pdl_launch_dependents();
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
       bool ok = true;
+      for (int s = 0; s < pre; ++s) {  // token halves of the stages started before the wait
+        const int u = u_begin + s;
+        const int kb = u - (u / KB) * KB;
+        tma_load_2d(smem + s * STAGE_BYTES + W_BYTES, &tmT, &full[s], kb * kBlockK, 0, pol_t);
+      }
+      p_issued = static_cast<uint32_t>(pre);
+      p_u = u_begin + pre;
+      p_stage = static_cast<uint32_t>(pre % STAGES);
+      p_phase = pre == STAGES ? 1u : 0u;
       for (; p_u < u_end; ++p_u) {
         if (!mbar_wait(&empty[p_stage], p_phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
         issue(p_u);

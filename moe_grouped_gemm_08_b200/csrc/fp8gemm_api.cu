@@ -24,6 +24,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 constexpr int kMaxDevices = 64;
+constexpr unsigned kKnownFlags = FG_FLAG_STATIC_B;
 constexpr int kMaxSwapMP = 128;
 constexpr int kCounterCapacity = 1 << 16;  // n-tiles of 128 rows: N <= 8,388,608 on the stream-K path
 
@@ -79,6 +80,18 @@ constexpr int kTiledStages = FG_TILED_STAGES;
 constexpr int kPairBN = FG_PAIR_BN;
 constexpr int kPairStages = FG_PAIR_STAGES;
 
+// tile width of the tiled and pair kernels: 0 automatic, else forced (fg_set_tile_n)
+std::atomic<int> g_tile_n{0};
+
+template <int BN>
+constexpr int tiled_stages() {
+  return BN == 128 ? 5 : (BN == 192 ? kTiledStages : 3);
+}
+template <int BN>
+constexpr int pair_stages() {
+  return BN == 192 ? kPairStages : 4;
+}
+
 template <int BN, int STAGES>
 constexpr size_t tiled_smem_bytes() {
   return 1024 /*alignment slack*/ + static_cast<size_t>(STAGES) * (kBlockM + BN) * kBlockK +
@@ -87,6 +100,8 @@ constexpr size_t tiled_smem_bytes() {
          4 * (fg::kMaskedMaxGroups + 1) /*masked prefix*/;
 }
 static_assert(tiled_smem_bytes<kTiledBN, kTiledStages>() <= 227 * 1024, "tiled kernel shared memory");
+static_assert(tiled_smem_bytes<128, tiled_stages<128>()>() <= 227 * 1024, "tiled kernel shared memory");
+static_assert(tiled_smem_bytes<256, tiled_stages<256>()>() <= 227 * 1024, "tiled kernel shared memory");
 
 template <int BN, int STAGES>
 constexpr size_t pair_smem_bytes() {
@@ -95,6 +110,7 @@ constexpr size_t pair_smem_bytes() {
          2 * (fg::kSaChunk * kBlockM + 2 * fg::kSaChunk) * 4 + 256 + 4 * (fg::kMaskedMaxGroups + 1);
 }
 static_assert(pair_smem_bytes<kPairBN, kPairStages>() <= 227 * 1024, "pair kernel shared memory");
+static_assert(pair_smem_bytes<256, pair_stages<256>()>() <= 227 * 1024, "pair kernel shared memory");
 
 template <int MP>
 constexpr int swap_stages() {
@@ -249,12 +265,11 @@ fg_status check_common(const void* A, const float* sfa, const void* B, const flo
   return FG_OK;
 }
 
-template <int MODE>
+template <int MODE, int BN>
 fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                     const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
                     int fmt_a, int fmt_b) {
-  constexpr int BN = kTiledBN;
-  constexpr int STAGES = kTiledStages;
+  constexpr int STAGES = tiled_stages<BN>();
   fg::TiledParams p;
   p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
   p.sfa = sfa;
@@ -310,6 +325,19 @@ fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* 
                                                               fg::kTiledThreads, fg::kTiledLaunchRegs);
 }
 
+// Tile width of the tiled kernel for a call: the forced width (fg_set_tile_n) if any, else 192.
+template <int MODE>
+fg_status dispatch_tiled(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                         const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
+                         int fmt_a, int fmt_b) {
+  const int bn = g_tile_n.load(std::memory_order_relaxed);
+  if (bn == 128)
+    return run_tiled<MODE, 128>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+  if (bn == 256)
+    return run_tiled<MODE, 256>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+  return run_tiled<MODE, kTiledBN>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+}
+
 // Largest number of CTA pairs of the pair kernel that can be resident at once (queried once per
 // device and kernel; clusters must fit inside a GPC, so this can be below #SMs / 2).
 template <auto KERNEL>
@@ -339,11 +367,10 @@ int pair_capacity(int sms, size_t smem) {
   return n;
 }
 
-template <int MODE>
+template <int MODE, int BN>
 fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
-  constexpr int BN = kPairBN;
-  constexpr int STAGES = kPairStages;
+  constexpr int STAGES = pair_stages<BN>();
   constexpr auto KERNEL = fg::fp8_gemm_pair_kernel<BN, STAGES, MODE>;
   constexpr size_t SMEM = pair_smem_bytes<BN, STAGES>();
   fg::TiledParams p;
@@ -389,6 +416,14 @@ fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B
   void* args[4] = {&mA, &mB, &mC, &p};
   return launch<KERNEL>(dim3(static_cast<unsigned>(2 * pairs)), SMEM, stream, args, fg::kTiledThreads,
                         fg::kTiledLaunchRegs);
+}
+
+template <int MODE>
+fg_status dispatch_pair(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                        const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
+  if (g_tile_n.load(std::memory_order_relaxed) == 256)
+    return run_pair<MODE, 256>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+  return run_pair<MODE, kPairBN>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
 }
 
 // Largest number of clusters of `size` CTAs of KERNEL that can be resident at once (clusters must
@@ -492,7 +527,7 @@ SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
 
 template <int MP>
 fg_status run_swap(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                   int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
+                   int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b, unsigned flags) {
   constexpr int STAGES = swap_stages<MP>();
   fg::SwapParams p;
   // swap-AB: the MMA's A operand is the weight tile (B of the GEMM), its B operand the tokens
@@ -511,6 +546,7 @@ fg_status run_swap(const Ctx* st, const void* A, const float* sfa, const void* B
   p.num_kb = (K + kBlockK - 1) / kBlockK;
   p.n_tiles = (N + kBlockM - 1) / kBlockM;
   p.debug_stall = g_debug_stall.load(std::memory_order_relaxed);
+  p.static_b = (flags & FG_FLAG_STATIC_B) ? 1 : 0;
   if (p.n_tiles > kCounterCapacity) return FG_ERR_UNSUPPORTED;
 
   CUtensorMap mW, mT;
@@ -593,6 +629,7 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   p.fmt_bits = 0;  // e4m3 x e4m3
   p.tile_aligned = 0;
   p.cluster = 1;
+  p.static_b = 0;
   if (p.n_tiles > kNoAllocCounters) return FG_ERR_UNSUPPORTED;
   // the counters must start at zero; the kernel leaves them at zero, but a call that gave up a
   // wait may not have, so clear the ones this call uses (a memset, no allocation)
@@ -676,6 +713,11 @@ uint64_t fg_launch_count(void) { return g_launches.load(); }
 
 int fg_debug_set_stall(int enable) { return g_debug_stall.exchange(enable ? 1 : 0); }
 
+int fg_set_tile_n(int bn) {
+  if (bn != 0 && bn != 128 && bn != 192 && bn != 256) return g_tile_n.load();
+  return g_tile_n.exchange(bn);
+}
+
 int fg_set_tiled_streamk(int overhead) { return g_tiled_sk.exchange(overhead < 0 ? -1 : overhead); }
 
 int fg_swap_plan(int M, int N, int K) {
@@ -722,8 +764,9 @@ static fg_status resolve_ctx(void* workspace, size_t workspace_bytes, Ctx* out) 
 }
 
 fg_status fp8_gemm_nt_ws(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
-                         int K, int fmt_a, int fmt_b, void* workspace, size_t workspace_bytes, void* stream) {
-  if (M < 0 || N < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
+                         int K, int fmt_a, int fmt_b, unsigned flags, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  if (M < 0 || N < 0 || !valid_formats(fmt_a, fmt_b) || (flags & ~kKnownFlags)) return FG_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return FG_OK;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
   if (s != FG_OK) return s;
@@ -738,17 +781,17 @@ fg_status fp8_gemm_nt_ws(const void* A, const float* sfa, const void* B, const f
   const bool swap = (path == 2) || (path == 0 && M <= kMaxSwapMP);
   if (swap) {
     if (M > kMaxSwapMP) return FG_ERR_UNSUPPORTED;
-    if (M <= 32) return run_swap<32>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b);
-    if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b);
-    return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b);
+    if (M <= 32) return run_swap<32>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b, flags);
+    if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b, flags);
+    return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b, flags);
   }
-  if (path == 3) return run_pair<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
-  return run_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
+  if (path == 3) return dispatch_pair<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
+  return dispatch_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
 }
 
 fg_status fp8_gemm_nt_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
                          int K, int fmt_a, int fmt_b, void* stream) {
-  return fp8_gemm_nt_ws(A, sfa, B, sfb, C, M, N, K, fmt_a, fmt_b, nullptr, 0, stream);
+  return fp8_gemm_nt_ws(A, sfa, B, sfb, C, M, N, K, fmt_a, fmt_b, 0u, nullptr, 0, stream);
 }
 
 fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const float* sfb, void* C, int M, int N,
@@ -758,8 +801,10 @@ fg_status fp8_gemm_nt(const void* A, const float* sfa, const void* B, const floa
 
 fg_status fp8_gemm_grouped_contiguous_ws(const void* A, const float* sfa, const void* B, const float* sfb,
                                          void* C, const int* m_indices, int M_total, int G, int N, int K, int fmt_a,
-                                         int fmt_b, void* workspace, size_t workspace_bytes, void* stream) {
-  if (M_total < 0 || N < 0 || G < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
+                                         int fmt_b, unsigned flags, void* workspace, size_t workspace_bytes,
+                                         void* stream) {
+  if (M_total < 0 || N < 0 || G < 0 || !valid_formats(fmt_a, fmt_b) || (flags & ~kKnownFlags))
+    return FG_ERR_INVALID_ARG;
   if (M_total == 0 || N == 0) return FG_OK;
   if (G == 0) return FG_ERR_INVALID_ARG;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
@@ -771,15 +816,15 @@ fg_status fp8_gemm_grouped_contiguous_ws(const void* A, const float* sfa, const 
   Ctx ctx;
   s = resolve_ctx(workspace, workspace_bytes, &ctx);
   if (s != FG_OK) return s;
-  return run_tiled<fg::kContiguous>(&ctx, A, sfa, B, sfb, C, m_indices, nullptr, M_total, G, N, K,
+  return dispatch_tiled<fg::kContiguous>(&ctx, A, sfa, B, sfb, C, m_indices, nullptr, M_total, G, N, K,
                                     static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
 }
 
 fg_status fp8_gemm_grouped_contiguous_ex(const void* A, const float* sfa, const void* B, const float* sfb,
                                          void* C, const int* m_indices, int M_total, int G, int N, int K, int fmt_a,
                                          int fmt_b, void* stream) {
-  return fp8_gemm_grouped_contiguous_ws(A, sfa, B, sfb, C, m_indices, M_total, G, N, K, fmt_a, fmt_b, nullptr, 0,
-                                        stream);
+  return fp8_gemm_grouped_contiguous_ws(A, sfa, B, sfb, C, m_indices, M_total, G, N, K, fmt_a, fmt_b, 0u, nullptr,
+                                        0, stream);
 }
 
 fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
@@ -789,8 +834,9 @@ fg_status fp8_gemm_grouped_contiguous(const void* A, const float* sfa, const voi
 
 fg_status fp8_gemm_grouped_masked_ws(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                                      const int* masked_m, int G, int Mmax, int N, int K, int fmt_a, int fmt_b,
-                                     void* workspace, size_t workspace_bytes, void* stream) {
-  if (G < 0 || Mmax < 0 || N < 0 || !valid_formats(fmt_a, fmt_b)) return FG_ERR_INVALID_ARG;
+                                     unsigned flags, void* workspace, size_t workspace_bytes, void* stream) {
+  if (G < 0 || Mmax < 0 || N < 0 || !valid_formats(fmt_a, fmt_b) || (flags & ~kKnownFlags))
+    return FG_ERR_INVALID_ARG;
   if (G == 0 || Mmax == 0 || N == 0) return FG_OK;
   fg_status s = check_common(A, sfa, B, sfb, C, N, K);
   if (s != FG_OK) return s;
@@ -803,16 +849,17 @@ fg_status fp8_gemm_grouped_masked_ws(const void* A, const float* sfa, const void
   s = resolve_ctx(workspace, workspace_bytes, &ctx);
   if (s != FG_OK) return s;
   if (g_dense_path.load() == 3)
-    return run_pair<fg::kMasked>(&ctx, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K, static_cast<cudaStream_t>(stream),
-                                 fmt_a, fmt_b);
-  return run_tiled<fg::kMasked>(&ctx, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
+    return dispatch_pair<fg::kMasked>(&ctx, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K,
+                                      static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
+  return dispatch_tiled<fg::kMasked>(&ctx, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
                                 static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
 }
 
 fg_status fp8_gemm_grouped_masked_ex(const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                                      const int* masked_m, int G, int Mmax, int N, int K, int fmt_a, int fmt_b,
                                      void* stream) {
-  return fp8_gemm_grouped_masked_ws(A, sfa, B, sfb, C, masked_m, G, Mmax, N, K, fmt_a, fmt_b, nullptr, 0, stream);
+  return fp8_gemm_grouped_masked_ws(A, sfa, B, sfb, C, masked_m, G, Mmax, N, K, fmt_a, fmt_b, 0u, nullptr, 0,
+                                     stream);
 }
 
 fg_status fp8_gemm_grouped_masked(const void* A, const float* sfa, const void* B, const float* sfb, void* C,

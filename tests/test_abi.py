@@ -129,11 +129,12 @@ def test_workspace_entry_points_check_arguments_first():
     if not torch.cuda.is_available():
         assert L.fg_workspace_bytes() == 0  # no fg_init on this device
         # arguments valid, no device state: not initialised, nothing launched
-        assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 0, 0, P16, 1 << 30, NULL) == 4
-    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 120, 0, 0, P16, 1 << 30, NULL) == 2   # K % 16
-    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 2, 0, P16, 1 << 30, NULL) == 1   # format
-    assert L.fp8_gemm_grouped_contiguous_ws(P16, P16, P16, P16, P16, NULL, 256, 2, 128, 128, 0, 0, P16, 1 << 30,
+        assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 0, 0, 1, P16, 1 << 30, NULL) == 4
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 120, 0, 0, 0, P16, 1 << 30, NULL) == 2   # K % 16
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 2, 0, 0, P16, 1 << 30, NULL) == 1   # format
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 64, 128, 128, 0, 0, 6, P16, 1 << 30, NULL) == 1   # flag
+    assert L.fp8_gemm_grouped_contiguous_ws(P16, P16, P16, P16, P16, NULL, 256, 2, 128, 128, 0, 0, 0, P16, 1 << 30,
                                             NULL) == 1
-    assert L.fp8_gemm_grouped_masked_ws(P16, P16, P16, P16, P16, P16, 2000, 64, 128, 128, 0, 0, P16, 1 << 30,
+    assert L.fp8_gemm_grouped_masked_ws(P16, P16, P16, P16, P16, P16, 2000, 64, 128, 128, 0, 0, 0, P16, 1 << 30,
                                         NULL) == 3
-    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 0, 128, 128, 0, 0, NULL, 0, NULL) == 0  # M = 0: no-op
+    assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 0, 128, 128, 0, 0, 0, NULL, 0, NULL) == 0  # M = 0: no-op
