@@ -604,6 +604,8 @@ def run_ours(args, rank, world, local):
         fg.set_tiled_streamk(args.tiled_streamk)
     if args.swap_schedule is not None:
         fg.set_swap_schedule(args.swap_schedule)
+    if args.tile_n is not None:
+        fg.set_tile_n(args.tile_n)
     stream = torch.cuda.Stream(device=dev)
     name, wl = workload_list(args.workload, args.shape)
     # The weights of a decode step are loaded once and never rewritten, so the dense calls declare
@@ -656,7 +658,8 @@ def run_ours(args, rank, world, local):
             "data": "synthetic",
             "config": dict(res["config"], parallelism=f"replicas x{world}", kernel_path=args.path,
                            tiled_streamk="library default" if args.tiled_streamk is None else args.tiled_streamk,
-                           swap_schedule="library default" if args.swap_schedule is None else args.swap_schedule),
+                           swap_schedule="library default" if args.swap_schedule is None else args.swap_schedule,
+                           tile_n="library default" if args.tile_n is None else args.tile_n),
             "hbm_gbs": res["hbm_gbs"], "shapes": res["shapes"], "shapes_timing": res["shapes_timing"],
             "roofline": res["roofline"],
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
@@ -666,12 +669,13 @@ def run_ours(args, rank, world, local):
         s, f, cores = time_oracle(cases, row_fraction=1.0)
         line["cpu_baseline"] = {"value": round(f / s / 1e12, 5), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                                 "sample": f"one full step of the {name} workload (every GEMM, all rows), {s:.1f} s"}
+    has_dense = any(c["kind"] == "dense" for c in cases)
     del cases
     torch.cuda.empty_cache()
 
     # the other configurations, timed the same way in the same process (same steps and warm-up)
     extra = [x for x in (args.also.split(",") if args.also else []) if x and x != name]
-    if args.static_b and not args.shape and any(c["kind"] == "dense" for c in cases):
+    if args.static_b and not args.shape and has_dense:
         extra = [name + ":ordered"] + extra
     if extra and not args.shape:
         line["workloads"] = {}
@@ -713,6 +717,8 @@ def main():
     ap.add_argument("--swap-schedule", type=int, default=None, choices=[-1, 0, 1, 2, 4, 8],
                     help="small-M kernel schedule (fg_set_swap_schedule): 0 automatic, -1 never the "
                          "cluster split, 1 whole tiles, 2/4/8 the cluster split with that many CTAs per tile")
+    ap.add_argument("--tile-n", type=int, default=None, choices=[0, 128, 192, 256],
+                    help="output tile width of the tiled / CTA-pair kernels (fg_set_tile_n): 0 automatic")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

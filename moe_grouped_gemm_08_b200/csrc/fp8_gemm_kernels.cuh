@@ -66,6 +66,11 @@ struct RegSplit {
 
 enum Mode : int { kDense = 0, kContiguous = 1, kMasked = 2 };
 
+// Promotion read pattern of the 256-wide tiles (promote_kblock's PIPE; a build-time knob).
+#ifndef FG_PIPE_256
+#define FG_PIPE_256 2
+#endif
+
 struct TiledParams {
   const float* sfa;
   const float* sfb;
@@ -359,8 +364,11 @@ __device__ __forceinline__ void store_scale_chunk(float* buf, int tid, const Sca
 // warp) hands the TMEM buffer back as soon as every chunk has landed in registers.
 // PIPE = false: every chunk is loaded, one wait, then all are added (one load round trip per K
 //   block; 32 NCH registers of slice).
-// PIPE = true: two chunks in flight at a time, chunk i+1 loading while chunk i is added (64
-//   registers of slice, so 128 x 256 tiles fit the register budget).
+// PIPE = 1: two 32-column chunks in flight at a time, chunk i+1 loading while chunk i is added
+//   (64 registers of slice, so 128 x 256 tiles fit the register budget);
+// PIPE = 2: the same with 16-column chunks (32 registers of slice);
+// PIPE = 3: two rounds of half the slice each (load, wait, add), no overlap inside the warp but
+//   only two load round trips per K block (NCH * 16 registers of slice).
 template <int NCH, int PIPE, typename Release>
 __device__ __forceinline__ void promote_kblock(uint32_t taddr, float2* acc, float s0, float s1, uint32_t hi_mask,
                                                Release&& release) {
@@ -382,6 +390,19 @@ __device__ __forceinline__ void promote_kblock(uint32_t taddr, float2* acc, floa
     release();
 #pragma unroll
     for (int i = 0; i < NCH; ++i) add(v[i], i, 32);
+  } else if constexpr (PIPE == 3) {
+    // two rounds of NCH/2 chunks: load, wait, add; the buffer is released after the second wait
+    static_assert(NCH % 2 == 0, "PIPE 3 needs an even chunk count");
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      uint32_t v[NCH / 2][32];
+#pragma unroll
+      for (int i = 0; i < NCH / 2; ++i) tmem_ld_32x32b_x32(taddr + 32 * (r * NCH / 2 + i), v[i]);
+      tmem_wait_ld();
+      if (r == 1) release();
+#pragma unroll
+      for (int i = 0; i < NCH / 2; ++i) add(v[i], r * NCH / 2 + i, 32);
+    }
   } else if constexpr (PIPE == 1) {
     uint32_t va[32], vb[32];
     tmem_ld_32x32b_x32(taddr, va);
@@ -429,7 +450,7 @@ constexpr int kStoreBoxBytes = 32 * 64;
 // BN = 192 keeps one slice read (three 32-column TMEM loads) per K block within the register
 // budget, so each TMEM buffer is handed back after a single load round trip; two buffers of 192
 // columns fit the 512 TMEM columns.
-template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? 2 : 0)>
+template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0)>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
@@ -811,7 +832,7 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 // tempty[b] of the leader counts the promotion warps of both CTAs.  Cluster barriers only right
 // after set-up and right before teardown, which every thread of both CTAs reaches; every other
 // wait is bounded.
-template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? 2 : 0)>
+template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0)>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmC, const TiledParams p) {

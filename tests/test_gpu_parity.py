@@ -75,6 +75,23 @@ def test_dense_odd_shapes(fg, M, N, K):
         close(run_dense(fg, case, path), ref, f"odd {M}x{N}x{K} path={path}")
 
 
+@pytest.mark.parametrize("bn", [128, 192, 256])
+@pytest.mark.parametrize("M,N,K", [(129, 520, 256), (300, 392, 1152), (513, 2048, 3072), (1000, 2112, 640)])
+def test_tile_widths(fg, bn, M, N, K):
+    """Every tile width of the tiled kernel (and 192 / 256 of the CTA pair), with the stream-K tail
+    forced, against the oracle: ragged M and N tails, partial waves."""
+    case = synth.dense_case(700 + M, M, N, K, row_scaled=True)
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
+    old = fg.set_tile_n(bn)
+    old_sk = fg.set_tiled_streamk(0)
+    try:
+        for path in ([1, 3] if bn != 128 else [1]):
+            close(run_dense(fg, case, path), ref, f"{M}x{N}x{K} bn={bn} path={path}")
+    finally:
+        fg.set_tile_n(old)
+        fg.set_tiled_streamk(old_sk)
+
+
 @pytest.mark.parametrize("w", workloads.decode_sweep(), ids=lambda w: w["name"])
 def test_decode_sweep_full(fg, w):
     case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"], row_scaled=True)
