@@ -169,18 +169,27 @@ def work_of(case):
     return flops, byt, M * K + N * K + 2 * M * N
 
 
-KERNEL_PATH = 0  # the kernel selection bench.py runs with (--path)
+_FG = None  # the binding, once run_ours has loaded it
 
 
 def kernel_name(case) -> str:
-    """The library kernel a case runs on under the selection KERNEL_PATH (fg_set_dense_path)."""
-    if case["kind"] == "contiguous":
-        return "fp8_gemm_tiled_kernel"
-    if KERNEL_PATH == 3:
-        return "fp8_gemm_pair_kernel"
-    if case["kind"] == "masked" or KERNEL_PATH == 1:
-        return "fp8_gemm_tiled_kernel"
-    return "fp8_gemm_swap_streamk_kernel" if (KERNEL_PATH == 2 or case["M"] <= 128) else "fp8_gemm_tiled_kernel"
+    """The library kernel a case runs on under the current settings (the library's own plan)."""
+    if case["kind"] == "masked":
+        plan = _FG.tile_plan("masked", case["Mmax"], case["N"], case["K"], case["G"])
+    elif case["kind"] == "contiguous":
+        plan = _FG.tile_plan("contiguous", case["M"], case["N"], case["K"], case["G"])
+    else:
+        plan = _FG.tile_plan("dense", case["M"], case["N"], case["K"], 1)
+    return {1: "fp8_gemm_tiled_kernel", 2: "fp8_gemm_swap_streamk_kernel",
+            3: "fp8_gemm_pair_kernel"}.get(plan // 1000, "unknown")
+
+
+def tile_width(case):
+    if case["kind"] == "dense" and case["M"] <= 128:
+        return None
+    layout = case["kind"]
+    M = case["Mmax"] if layout == "masked" else case["M"]
+    return _FG.tile_plan(layout, M, case["N"], case["K"], case.get("G", 1)) % 1000
 
 
 def upload(case, dev):
@@ -547,6 +556,8 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local, static_b=Fal
         if kernel_name(c) == "fp8_gemm_swap_streamk_kernel":
             plan = fg.swap_plan(c["M"], c["N"], c["K"])
             shapes[-1]["schedule"] = {0: "stream-K", 1: "whole tiles"}.get(plan, f"cluster x{plan}")
+        else:
+            shapes[-1]["tile_n"] = tile_width(c)
         sum_ms_all += ms
         if kernel_name(c) == dom:
             sum_bytes_dom += wk[1]
@@ -597,8 +608,8 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     fg.init(local)
-    global KERNEL_PATH
-    KERNEL_PATH = args.path
+    global _FG
+    _FG = fg
     fg.set_dense_path(args.path)
     if args.tiled_streamk is not None:
         fg.set_tiled_streamk(args.tiled_streamk)
@@ -606,6 +617,8 @@ def run_ours(args, rank, world, local):
         fg.set_swap_schedule(args.swap_schedule)
     if args.tile_n is not None:
         fg.set_tile_n(args.tile_n)
+    if args.swap_kps is not None:
+        fg.set_swap_kps(args.swap_kps)
     stream = torch.cuda.Stream(device=dev)
     name, wl = workload_list(args.workload, args.shape)
     # The weights of a decode step are loaded once and never rewritten, so the dense calls declare
@@ -659,7 +672,8 @@ def run_ours(args, rank, world, local):
             "config": dict(res["config"], parallelism=f"replicas x{world}", kernel_path=args.path,
                            tiled_streamk="library default" if args.tiled_streamk is None else args.tiled_streamk,
                            swap_schedule="library default" if args.swap_schedule is None else args.swap_schedule,
-                           tile_n="library default" if args.tile_n is None else args.tile_n),
+                           tile_n="library default" if args.tile_n is None else args.tile_n,
+                           swap_kps="library default" if args.swap_kps is None else args.swap_kps),
             "hbm_gbs": res["hbm_gbs"], "shapes": res["shapes"], "shapes_timing": res["shapes_timing"],
             "roofline": res["roofline"],
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
@@ -719,6 +733,8 @@ def main():
                          "cluster split, 1 whole tiles, 2/4/8 the cluster split with that many CTAs per tile")
     ap.add_argument("--tile-n", type=int, default=None, choices=[0, 128, 192, 256],
                     help="output tile width of the tiled / CTA-pair kernels (fg_set_tile_n): 0 automatic")
+    ap.add_argument("--swap-kps", type=int, default=None, choices=[0, 1, 2],
+                    help="K blocks per ring stage of the small-M kernel (fg_set_swap_kps): 0 automatic")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

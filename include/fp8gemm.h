@@ -239,21 +239,31 @@ fg_status fg_get_device_status(void* stream);
 const char* fg_status_string(fg_status status);
 
 /* Kernel selection, process-wide: 0 = automatic (dense M <= 128 takes the
- * swap-AB kernel, scheduled as fg_set_swap_schedule says, everything else the
- * one-CTA tiled kernel), 1 = the one-CTA tiled kernel for every dense call, 2 =
- * always the swap-AB kernel for dense calls (requires M <= 128), 3 = the CTA-pair
- * kernel (tcgen05 cta_group::2,
- * 256-row tiles over two SMs) for dense and masked calls.  The contiguous layout
- * always takes the one-CTA tiled kernel.  Returns the previous value; an unknown
- * value is ignored. */
+ * swap-AB kernel, scheduled as fg_set_swap_schedule says; everything else follows
+ * the tile table -- see fg_tile_plan), 1 = the one-CTA tiled kernel for every
+ * dense, contiguous and masked call, 2 = always the swap-AB kernel for dense calls
+ * (requires M <= 128), 3 = the CTA-pair kernel (tcgen05 cta_group::2, 256-row
+ * tiles over two SMs) for dense and masked calls.  The contiguous layout never
+ * takes the CTA pair.  Returns the previous value; an unknown value is ignored. */
 int fg_set_dense_path(int path);
 
 /* Output tile width (columns of N per tile) of the tiled and CTA-pair kernels, process-wide:
- * 0 (default) = automatic, or 128, 192 or 256 to force a width (the CTA-pair kernel has
+ * 0 (default) = the tile table, or 128, 192 or 256 to force a width (the CTA-pair kernel has
  * 192 and 256; it takes 192 for a forced 128).  Widths other than these are ignored.
  * Results are identical in every width up to fp32 summation order of split tiles.
  * Returns the previous value. */
 int fg_set_tile_n(int bn);
+
+/* The kernel and tile width a call of this shape takes on the current device under the
+ * current settings, as kernel * 1000 + width: 1xxx the one-CTA tiled kernel, 3xxx the
+ * CTA pair, 2000 the small-M swap-AB kernel (dense, M <= 128).  layout: 0 dense, 1
+ * contiguous (M = all rows), 2 masked (M = Mmax); G = 1 for dense.  The tile table
+ * (automatic settings): N <= 128 -> 128-wide tiles, N <= 192 -> 192, otherwise 256; dense
+ * calls take the CTA pair unless its last wave of 256 x 256 tiles would hold at most a
+ * quarter of the SM pairs (then the one-CTA kernel, whose stream-K tail splits that wave),
+ * contiguous and masked calls the one-CTA kernel.  -1 for invalid arguments or a device
+ * without fg_init.  Launches nothing. */
+int fg_tile_plan(int layout, int M, int N, int K, int G);
 
 /* Stream-K tail of the tiled kernel (dense M > 128, contiguous, masked), process-wide.
  * The tiles are walked whole in waves over the SMs; when the last wave is partial
@@ -278,6 +288,15 @@ int fg_set_tiled_streamk(int overhead);
  * wherever it is possible.  Other values are ignored.  All schedules sum in a fixed
  * order.  Returns the previous value. */
 int fg_set_swap_schedule(int schedule);
+
+/* K blocks per ring stage of the small-M kernel, process-wide: 0 (default) = automatic -- 2
+ * when K is a multiple of 128 with at least four K blocks, each weight and token copy then
+ * moving two K blocks at once (a CTA's copy rate is bounded by the number of copies in flight
+ * more than by their size) -- else 1; 1 forces single K blocks; 2 forces pairs wherever K is a
+ * multiple of 128.  Any other value is ignored.  Results agree to fp32 summation order (split
+ * points of the K range move to pair boundaries).
+ * Returns the previous value. */
+int fg_set_swap_kps(int kps);
 
 /* The schedule the small-M kernel takes for a dense call of this shape on the current
  * device under the current setting: S (2, 4 or 8) for the cluster split, 1 for whole

@@ -72,10 +72,14 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_set_dense_path.restype = _int
     l.fg_debug_set_stall.argtypes = [_int]
     l.fg_debug_set_stall.restype = _int
+    l.fg_tile_plan.argtypes = [_int, _int, _int, _int, _int]
+    l.fg_tile_plan.restype = _int
     l.fg_set_tile_n.argtypes = [_int]
     l.fg_set_tile_n.restype = _int
     l.fg_set_tiled_streamk.argtypes = [_int]
     l.fg_set_tiled_streamk.restype = _int
+    l.fg_set_swap_kps.argtypes = [_int]
+    l.fg_set_swap_kps.restype = _int
     l.fg_set_swap_schedule.argtypes = [_int]
     l.fg_set_swap_schedule.restype = _int
     l.fg_swap_plan.argtypes = [_int, _int, _int]
@@ -158,6 +162,13 @@ def set_tile_n(bn: int) -> int:
     return int(_lib.fg_set_tile_n(int(bn)))
 
 
+def tile_plan(layout: str, M: int, N: int, K: int, G: int = 1) -> int:
+    """kernel * 1000 + tile width a call takes (1xxx one-CTA tiled, 3xxx CTA pair, 2000 swap-AB);
+    layout "dense", "contiguous" or "masked"; -1 if not applicable."""
+    code = {"dense": 0, "contiguous": 1, "masked": 2}[layout]
+    return int(_lib.fg_tile_plan(code, int(M), int(N), int(K), int(G)))
+
+
 def set_tiled_streamk(overhead: int) -> int:
     """Stream-K tail of the tiled kernel: split the last partial wave when its cost (its units +
     `overhead` K blocks + 2.4 per piece summed) is at most one tile (default 18; 0 whenever the last
@@ -169,6 +180,12 @@ def set_swap_schedule(schedule: int) -> int:
     """Small-M kernel schedule: 0 automatic, -1 never the cluster split, 1 whole tiles, 2/4/8 the
     cluster split with that many CTAs per weight tile wherever possible. Returns the old value."""
     return int(_lib.fg_set_swap_schedule(int(schedule)))
+
+
+def set_swap_kps(kps: int) -> int:
+    """K blocks per ring stage of the small-M kernel: 0 automatic (2 when K % 128 == 0), 1 or 2.
+    Returns the old value."""
+    return int(_lib.fg_set_swap_kps(int(kps)))
 
 
 def swap_plan(M: int, N: int, K: int) -> int:

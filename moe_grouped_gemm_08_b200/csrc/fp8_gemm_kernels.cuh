@@ -1192,19 +1192,27 @@ __device__ __forceinline__ void cluster_reduce_store(const SwapParams& p, uint32
   }
 }
 
-template <int MP, int STAGES>
+// KPS: K blocks per ring stage (and per unit of work).  KPS = 1 loads each K block's weight and
+// token tiles with 2-D TMA copies; KPS > 1 (K a multiple of 128) loads KPS consecutive K blocks
+// of each with one 3-D copy over the view {128 bytes, rows, K blocks} (strides K and 128 bytes),
+// which lands as KPS tiles one after the other -- the layout KPS 2-D copies would give -- so a
+// CTA streams its weights with half (a third, ...) of the copy operations: a CTA's copy rate is
+// bounded by the number of copies in flight, not by their size, up to ~32 KB per copy.
+template <int MP, int STAGES, int KPS = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_swap_streamk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
                                  const SwapParams p) {
   static_assert(MP == 32 || MP == 64 || MP == 128, "MP");
-  constexpr int W_BYTES = kBlockM * kBlockK;  // 128 weight rows
-  constexpr int T_BYTES = MP * kBlockK;       // MP token rows
-  constexpr int STAGE_BYTES = W_BYTES + T_BYTES;
+  static_assert(KPS == 1 || KPS == 2 || KPS == 4, "KPS");
+  constexpr int W_BYTES = kBlockM * kBlockK;  // one K block of 128 weight rows
+  constexpr int T_BYTES = MP * kBlockK;       // one K block of MP token rows
+  constexpr int STAGE_BYTES = KPS * (W_BYTES + T_BYTES);  // [KPS weight tiles][KPS token tiles]
   constexpr int NUM_TBUF = 4;
   constexpr uint32_t TMEM_COLS = (NUM_TBUF * MP) < 32 ? 32 : NUM_TBUF * MP;
   constexpr int COLS = MP / 2;                // token columns per promotion thread
   constexpr int NPROMO = kPromoWarps * 32;
-  constexpr int SCALE_CAP = kSwapScaleBytes / (4 * MP);  // units whose scales fit in shared memory
+  constexpr int SCALE_SLOTS = kSwapScaleBytes / (4 * MP);  // K blocks whose scales fit in shared memory
+  constexpr int SCALE_CAP = SCALE_SLOTS / KPS;              // units whose scales fit
   constexpr int F4 = MP * kBlockM / 4 / NPROMO;          // float4 of a partial tile per thread
   constexpr int PPR = (16 / F4) < 1 ? 1 : 16 / F4;       // partials read per round in the fix-up
   constexpr int RING_SLOTS = (STAGES * STAGE_BYTES) / (MP * kBlockM * 4);  // partials the idle ring holds
@@ -1214,8 +1222,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);
   __nv_bfloat16* s_c = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * STAGE_BYTES);  // [MP][128]
-  float* s_scale = reinterpret_cast<float*>(s_c + MP * kBlockM);                        // [SCALE_CAP][MP]
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + SCALE_CAP * MP);
+  float* s_scale = reinterpret_cast<float*>(s_c + MP * kBlockM);                        // [SCALE_SLOTS][MP]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + SCALE_SLOTS * MP);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + NUM_TBUF;
@@ -1228,7 +1236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int P = gridDim.x;
-  const int KB = p.num_kb;
+  const int NKB = p.num_kb;                 // K blocks
+  const int KB = (NKB + KPS - 1) / KPS;     // units (groups of KPS K blocks) per tile
   const int U = p.n_tiles * KB;
   // unit range: stream-K (even split of the units, tiles split between CTAs) or, when the host
   // finds whole tiles cheaper, tile-aligned (an even split of the tiles; no tile is split)
@@ -1243,6 +1252,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     : p.tile_aligned
                         ? static_cast<int>(static_cast<long long>(blockIdx.x + 1) * p.n_tiles / P) * KB
                         : sk_begin(blockIdx.x + 1, P, U);
+  // K blocks of unit u (the last unit of a tile may hold fewer than KPS)
+  auto unit_kblocks = [&](int u) {
+    const int kb0 = (u - (u / KB) * KB) * KPS;
+    return (NKB - kb0) < KPS ? (NKB - kb0) : KPS;
+  };
 
   const uint64_t pol_w = l2_policy_evict_first();  // each weight byte is read once
   const uint64_t pol_t = l2_policy_evict_last();   // tokens are re-read by every CTA
@@ -1250,14 +1264,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   int p_u = u_begin;
   uint32_t p_stage = 0, p_phase = 0;
   uint32_t p_issued = 0;
-  auto issue = [&](int u) {
+  // weight / token copies of unit u into stage `st` (a K-block group: first K block kb)
+  auto load_w = [&](int u, int st) {
     const int t = u / KB;
-    const int kb = u - t * KB;
+    const int kb = (u - t * KB) * KPS;
     FG_DCHECK(t >= 0 && t < p.n_tiles && t * kBlockM < p.N && kb * kBlockK < p.K, p.status);
-    uint8_t* sw = smem + p_stage * STAGE_BYTES;
-    mbar_arrive_expect_tx(&full[p_stage], STAGE_BYTES);
-    tma_load_2d(sw, &tmW, &full[p_stage], kb * kBlockK, t * kBlockM, pol_w);
-    tma_load_2d(sw + W_BYTES, &tmT, &full[p_stage], kb * kBlockK, 0, pol_t);
+    if constexpr (KPS == 1) tma_load_2d(smem + st * STAGE_BYTES, &tmW, &full[st], kb * kBlockK, t * kBlockM, pol_w);
+    else tma_load_3d(smem + st * STAGE_BYTES, &tmW, &full[st], 0, t * kBlockM, kb, pol_w);
+  };
+  auto load_t = [&](int u, int st) {
+    const int kb = (u - (u / KB) * KB) * KPS;
+    if constexpr (KPS == 1) tma_load_2d(smem + st * STAGE_BYTES + W_BYTES, &tmT, &full[st], kb * kBlockK, 0, pol_t);
+    else tma_load_3d(smem + st * STAGE_BYTES + KPS * W_BYTES, &tmT, &full[st], 0, 0, kb, pol_t);
+  };
+  auto issue = [&](int u) {
+    mbar_arrive_expect_tx(&full[p_stage], STAGE_BYTES);  // whole boxes, also where they pass K
+    load_w(u, p_stage);
+    load_t(u, p_stage);
     ++p_issued;
     if (++p_stage == STAGES) { p_stage = 0; p_phase ^= 1u; }
   };
@@ -1284,12 +1307,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (p.static_b && warp == kProducerWarp && lane == 0) {
     pre = (u_end - u_begin) < STAGES ? (u_end - u_begin) : STAGES;
     for (int s = 0; s < pre; ++s) {
-      const int u = u_begin + s;
-      const int t = u / KB;
-      const int kb = u - t * KB;
-      FG_DCHECK(t >= 0 && t < p.n_tiles && t * kBlockM < p.N && kb * kBlockK < p.K, p.status);
       mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-      tma_load_2d(smem + s * STAGE_BYTES, &tmW, &full[s], kb * kBlockK, t * kBlockM, pol_w);
+      load_w(u_begin + s, s);
     }
   }
   // Everything above overlaps the previous kernel's tail; from here on global memory is touched
@@ -1300,11 +1319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp) {
     if (lane == 0) {
       bool ok = true;
-      for (int s = 0; s < pre; ++s) {  // token halves of the stages started before the wait
-        const int u = u_begin + s;
-        const int kb = u - (u / KB) * KB;
-        tma_load_2d(smem + s * STAGE_BYTES + W_BYTES, &tmT, &full[s], kb * kBlockK, 0, pol_t);
-      }
+      for (int s = 0; s < pre; ++s) load_t(u_begin + s, s);  // token halves of the early stages
       p_issued = static_cast<uint32_t>(pre);
       p_u = u_begin + pre;
       p_stage = static_cast<uint32_t>(pre % STAGES);
@@ -1324,21 +1339,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Failure-injection hook for tests: mma_done completes its first phase only with the commit
       // below, so this bounded wait runs out, raises the abort flag and exercises the abort path.
       if (p.debug_stall) mbar_wait(mma_done, 0, abort_flag, kWaitLimitNs);
-      for (int u = u_begin; u < u_end; ++u) {
+      bool ok = true;
+      for (int u = u_begin; u < u_end && ok; ++u) {
         if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
-        if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + tb * MP;
-        const uint32_t sw = smem_addr(smem + stage * STAGE_BYTES);
-        const uint64_t adesc = smem_desc_k128_sw128(sw);
-        const uint64_t bdesc = smem_desc_k128_sw128(sw + W_BYTES);
+        const int nk = unit_kblocks(u);
+        for (int i = 0; i < nk; ++i) {  // one TMEM partial per K block
+          if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t d = tmem_base + tb * MP;
+          const uint32_t sw = smem_addr(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = smem_desc_k128_sw128(sw + i * W_BYTES);
+          const uint64_t bdesc = smem_desc_k128_sw128(sw + KPS * W_BYTES + i * T_BYTES);
 #pragma unroll
-        for (int j = 0; j < kBlockK / 32; ++j)
-          mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
-        mma_commit(&empty[stage]);
-        mma_commit(&tfull[tb]);
+          for (int j = 0; j < kBlockK / 32; ++j)
+            mma_f8(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
+          if (i == nk - 1) mma_commit(&empty[stage]);
+          mma_commit(&tfull[tb]);
+          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+        }
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-        if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
       }
       mma_commit(mma_done);
       mbar_drain(mma_done, 0);
@@ -1382,66 +1401,73 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int j = 0; j < COLS; ++j) acc[j] = 0.0f;
 
-      for (int kb = kb0; kb < kb1; ++kb) {
-        const int uu = tu0 + kb;
+      for (int kb = kb0; kb < kb1 && ok; ++kb) {
+        const int uu = tu0 + kb;  // unit (group of KPS K blocks)
         if (uu >= chunk_end) {
-          // combined scales sfa[kb][m] * sfb[t][kb] of the next SCALE_CAP units (zero past M);
-          // thread tid owns column tid % MP of units tid / MP + r * (256 / MP), and every load
-          // of the chunk is issued before the first product is formed
+          // combined scales sfa[k][m] * sfb[t][k] of the K blocks of the next SCALE_CAP units (zero
+          // past M and past the last K block); slot sl = KPS * (unit - chunk_base) + i holds K
+          // block i of the unit.  Thread tid owns column tid % MP of slots tid / MP + r * (256 /
+          // MP), and every load of the chunk is issued before the first product is formed
           if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
           chunk_base = uu;
           chunk_end = (u_end < uu + SCALE_CAP) ? u_end : uu + SCALE_CAP;
-          constexpr int STEP = NPROMO / MP;  // units per pass of all threads
-          constexpr int ITER = SCALE_CAP / STEP;
+          constexpr int STEP = NPROMO / MP;  // slots per pass of all threads
+          constexpr int ITER = SCALE_SLOTS / STEP;
           const int mm = tid % MP;
-          const int v0 = chunk_base + tid / MP;
           float a[ITER], b[ITER];
-          // each unit's (tile, K block) is computed on its own, so that no load waits for an index
+          // each slot's (tile, K block) is computed on its own, so that no load waits for an index
           // chain: all of a thread's scale loads are in flight together
 #pragma unroll
           for (int r = 0; r < ITER; ++r) {
             a[r] = 0.0f;
             b[r] = 0.0f;
-            const int v = v0 + r * STEP;
+            const int sl = tid / MP + r * STEP;
+            const int v = chunk_base + sl / KPS;
             if (v < chunk_end) {
               const int vt = v / KB;
-              const int vkb = v - vt * KB;
-              if (mm < p.M) a[r] = __ldg(p.sfa + static_cast<size_t>(vkb) * p.ld + mm);
-              b[r] = __ldg(p.sfb + static_cast<size_t>(vt) * KB + vkb);
+              const int vkb = (v - vt * KB) * KPS + sl % KPS;
+              if (vkb < NKB) {
+                if (mm < p.M) a[r] = __ldg(p.sfa + static_cast<size_t>(vkb) * p.ld + mm);
+                b[r] = __ldg(p.sfb + static_cast<size_t>(vt) * NKB + vkb);
+              }
             }
           }
 #pragma unroll
           for (int r = 0; r < ITER; ++r) s_scale[(tid / MP + r * STEP) * MP + mm] = a[r] * b[r];
           if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
         }
-        if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t taddr = tmem_base + lane_off + tb * MP + h * COLS;
-        uint32_t v[COLS];
-        if constexpr (COLS == 16) {
-          uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
-          tmem_ld_32x32b_x16(taddr, r16);
-        } else {
+        const int nk = unit_kblocks(uu);
+        for (int i = 0; i < nk; ++i) {
+          if (!mbar_wait(&tfull[tb], tphase, abort_flag, kWaitLimitNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + lane_off + tb * MP + h * COLS;
+          uint32_t v[COLS];
+          if constexpr (COLS == 16) {
+            uint32_t (&r16)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+            tmem_ld_32x32b_x16(taddr, r16);
+          } else {
 #pragma unroll
-          for (int c0 = 0; c0 < COLS; c0 += 32) {
-            uint32_t (&r32)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + c0);
-            tmem_ld_32x32b_x32(taddr + c0, r32);
+            for (int c0 = 0; c0 < COLS; c0 += 32) {
+              uint32_t (&r32)[32] = *reinterpret_cast<uint32_t(*)[32]>(v + c0);
+              tmem_ld_32x32b_x32(taddr + c0, r32);
+            }
           }
-        }
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[tb]);
-        const float4* sc4 = reinterpret_cast<const float4*>(s_scale + (uu - chunk_base) * MP + h * COLS);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[tb]);
+          const float4* sc4 =
+              reinterpret_cast<const float4*>(s_scale + ((uu - chunk_base) * KPS + i) * MP + h * COLS);
 #pragma unroll
-        for (int j = 0; j < COLS; j += 4) {
-          const float4 s4 = sc4[j / 4];
-          acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), s4.x, acc[j + 0]);
-          acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), s4.y, acc[j + 1]);
-          acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), s4.z, acc[j + 2]);
-          acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), s4.w, acc[j + 3]);
+          for (int j = 0; j < COLS; j += 4) {
+            const float4 s4 = sc4[j / 4];
+            acc[j + 0] = fmaf(__uint_as_float(v[j + 0]), s4.x, acc[j + 0]);
+            acc[j + 1] = fmaf(__uint_as_float(v[j + 1]), s4.y, acc[j + 1]);
+            acc[j + 2] = fmaf(__uint_as_float(v[j + 2]), s4.z, acc[j + 2]);
+            acc[j + 3] = fmaf(__uint_as_float(v[j + 3]), s4.w, acc[j + 3]);
+          }
+          if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
         }
-        if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
       }
       if (!ok) break;
 

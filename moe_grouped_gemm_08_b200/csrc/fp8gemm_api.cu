@@ -112,16 +112,24 @@ constexpr size_t pair_smem_bytes() {
 static_assert(pair_smem_bytes<kPairBN, kPairStages>() <= 227 * 1024, "pair kernel shared memory");
 static_assert(pair_smem_bytes<256, pair_stages<256>()>() <= 227 * 1024, "pair kernel shared memory");
 
-template <int MP>
+// Ring stages of the small-M kernel by MP and K blocks per stage (KPS): about 192 KB of ring.
+template <int MP, int KPS = 1>
 constexpr int swap_stages() {
-  return MP == 128 ? 5 : (MP == 64 ? 8 : 10);
+  return KPS == 1 ? (MP == 128 ? 5 : (MP == 64 ? 8 : 10)) : (MP == 128 ? 2 : (MP == 64 ? 4 : 5));
 }
 
-template <int MP, int STAGES>
+template <int MP, int STAGES, int KPS = 1>
 constexpr size_t swap_smem_bytes() {
-  return 1024 + static_cast<size_t>(STAGES) * (kBlockM + MP) * kBlockK + MP * kBlockM * 2 /*C staging*/ +
+  return 1024 + static_cast<size_t>(STAGES) * KPS * (kBlockM + MP) * kBlockK + MP * kBlockM * 2 /*C staging*/ +
          fg::kSwapScaleBytes /*combined scales*/ + 256 /*barriers*/;
 }
+static_assert(swap_smem_bytes<32, swap_stages<32, 2>(), 2>() <= 227 * 1024, "swap kernel shared memory");
+static_assert(swap_smem_bytes<64, swap_stages<64, 2>(), 2>() <= 227 * 1024, "swap kernel shared memory");
+static_assert(swap_smem_bytes<128, swap_stages<128, 2>(), 2>() <= 227 * 1024, "swap kernel shared memory");
+
+// K blocks per stage of the small-M kernel: 0 automatic (2 when K is a multiple of 128, else 1),
+// or 1 / 2 forced (2 only where K allows it; fg_set_swap_kps)
+std::atomic<int> g_swap_kps{0};
 
 int current_device() {
   int dev = -1;
@@ -189,6 +197,22 @@ bool encode_bf16_store_map(CUtensorMap* map, void* base, uint64_t N, uint64_t ro
   cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, three_d ? 3 : 2, base, dims, strides, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D view of a K-major e4m3 matrix [rows, K] (K a multiple of 128) as {128 bytes of a K block,
+// rows, K blocks} with strides {K, 128}: a box {128, box_rows, kps} is kps consecutive K blocks of
+// box_rows rows, laid out in shared memory as kps tiles of box_rows x 128 bytes one after the other
+// (each 128-byte swizzled like a 2-D copy of it).
+bool encode_fp8_map_kblocks(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows,
+                            uint32_t kps) {
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBlockK), rows, K / kBlockK};
+  cuuint64_t strides[2] = {K, static_cast<cuuint64_t>(kBlockK)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockK), box_rows, kps};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -325,19 +349,6 @@ fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* 
                                                               fg::kTiledThreads, fg::kTiledLaunchRegs);
 }
 
-// Tile width of the tiled kernel for a call: the forced width (fg_set_tile_n) if any, else 192.
-template <int MODE>
-fg_status dispatch_tiled(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                         const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
-                         int fmt_a, int fmt_b) {
-  const int bn = g_tile_n.load(std::memory_order_relaxed);
-  if (bn == 128)
-    return run_tiled<MODE, 128>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
-  if (bn == 256)
-    return run_tiled<MODE, 256>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
-  return run_tiled<MODE, kTiledBN>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
-}
-
 // Largest number of CTA pairs of the pair kernel that can be resident at once (queried once per
 // device and kernel; clusters must fit inside a GPC, so this can be below #SMs / 2).
 template <auto KERNEL>
@@ -418,12 +429,58 @@ fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B
                         fg::kTiledLaunchRegs);
 }
 
+// Kernel and output tile width of a call of the tiled family (dense M > 128, contiguous, masked).
+// The tile table (measured on B200, prefill / contiguous / masked benchmark shapes): 256-wide tiles
+// run 8-13% faster than 192-wide ones (one TMEM round trip per K block stays within the register
+// budget with pipelined TMEM reads, and each K block's copies carry more bytes); the CTA pair
+// (256 x 256 per two SMs, each SM loading half of the weight tile) is best for dense calls unless
+// its last wave is nearly empty -- it has no stream-K tail, the one-CTA kernel does -- and cannot
+// serve the contiguous layout (a 256-row tile may straddle two experts).  Narrow N takes narrower
+// tiles.  fg_set_dense_path (1 one-CTA, 3 pair) and fg_set_tile_n override the table.
+struct TilePlan {
+  int kernel;  // 1: one-CTA tiled kernel, 3: CTA-pair kernel
+  int bn;      // 128, 192 or 256
+};
+
+TilePlan tile_plan(int mode, int M, int N, int G, int sms) {
+  const int path = g_dense_path.load(std::memory_order_relaxed);
+  const int forced = g_tile_n.load(std::memory_order_relaxed);
+  TilePlan t;
+  if (N <= 128) t = {1, 128};
+  else if (N <= 192) t = {1, 192};
+  else if (mode != fg::kDense) t = {1, 256};
+  else {
+    const long long pair_tiles = static_cast<long long>((M + 255) / 256) * ((N + 255) / 256);
+    const int pairs = sms / 2 > 0 ? sms / 2 : 1;
+    const long long rem = pair_tiles % pairs;
+    // a last wave holding at most a quarter of the pairs: the one-CTA kernel's stream-K tail wins
+    t = (rem != 0 && rem * 4 <= pairs) ? TilePlan{1, 256} : TilePlan{3, 256};
+    (void)G;
+  }
+  if (path == 1) t.kernel = 1;
+  if (path == 3 && mode != fg::kContiguous) t.kernel = 3;
+  if (forced != 0) t.bn = forced;
+  if (t.kernel == 3 && t.bn != 256) t.bn = 192;  // the pair kernel has 192 and 256
+  return t;
+}
+
 template <int MODE>
-fg_status dispatch_pair(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                        const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
-  if (g_tile_n.load(std::memory_order_relaxed) == 256)
-    return run_pair<MODE, 256>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
-  return run_pair<MODE, kPairBN>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+fg_status dispatch_tiled(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                         const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
+                         int fmt_a, int fmt_b) {
+  const TilePlan t = tile_plan(MODE, M, N, G, st->sms);
+  if (t.kernel == 3 && MODE != fg::kContiguous) {
+    if (t.bn == 256)
+      return run_pair<MODE == fg::kContiguous ? fg::kDense : MODE, 256>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K,
+                                                                         stream, fmt_a, fmt_b);
+    return run_pair<MODE == fg::kContiguous ? fg::kDense : MODE, kPairBN>(st, A, sfa, B, sfb, C, masked_m, M, G, N,
+                                                                            K, stream, fmt_a, fmt_b);
+  }
+  if (t.bn == 128)
+    return run_tiled<MODE, 128>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+  if (t.bn == 256)
+    return run_tiled<MODE, 256>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+  return run_tiled<MODE, kTiledBN>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
 }
 
 // Largest number of clusters of `size` CTAs of KERNEL that can be resident at once (clusters must
@@ -486,17 +543,19 @@ struct SwapChoice {
 #ifndef FG_SWAP_STREAMK_UNITS
 #define FG_SWAP_STREAMK_UNITS 16
 #endif
-template <int MP>
-SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
-  constexpr int STAGES = swap_stages<MP>();
-  constexpr auto KERNEL = fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>;
-  constexpr size_t SMEM = swap_smem_bytes<MP, STAGES>();
+// Units are groups of KPS K blocks (the last of a tile may be shorter); costs are in K blocks.
+template <int MP, int KPS = 1>
+SwapChoice swap_choose(int sms, int n_tiles, int num_kb_blocks) {
+  constexpr int STAGES = swap_stages<MP, KPS>();
+  constexpr auto KERNEL = fg::fp8_gemm_swap_streamk_kernel<MP, STAGES, KPS>;
+  constexpr size_t SMEM = swap_smem_bytes<MP, STAGES, KPS>();
   constexpr long long kSplitOverheadUnits = FG_SPLIT_OVERHEAD_UNITS;
+  const int num_kb = (num_kb_blocks + KPS - 1) / KPS;  // units per tile
   SwapChoice c;
   const long long units = static_cast<long long>(n_tiles) * num_kb;
   c.grid = static_cast<int>(units < sms ? units : sms);
-  const long long aligned_units = (n_tiles + sms - 1) / sms * static_cast<long long>(num_kb);
-  const long long split_units = (units + c.grid - 1) / c.grid;
+  const long long aligned_units = (n_tiles + sms - 1) / sms * static_cast<long long>(num_kb_blocks);
+  const long long split_units = (units + c.grid - 1) / c.grid * KPS;
   c.tile_aligned = (n_tiles >= sms && aligned_units <= split_units + kSplitOverheadUnits) ? 1 : 0;
   if (c.tile_aligned) c.grid = sms;
   c.cluster = 1;
@@ -511,7 +570,7 @@ SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
     for (int S : {8, 4, 2}) {
       if (sched > 0 && S != sched) continue;
       if (S > num_kb || n_tiles > cluster_capacity<KERNEL>(S, fg::kThreads, SMEM)) continue;
-      const long long cost = (num_kb + S - 1) / S + FG_SWAP_CLUSTER_UNITS;
+      const long long cost = (num_kb + S - 1) / S * KPS + FG_SWAP_CLUSTER_UNITS;
       if (sched > 0 || cost < best) {
         best = cost;
         c.cluster = S;
@@ -525,10 +584,10 @@ SwapChoice swap_choose(int sms, int n_tiles, int num_kb) {
   return c;
 }
 
-template <int MP>
-fg_status run_swap(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
-                   int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b, unsigned flags) {
-  constexpr int STAGES = swap_stages<MP>();
+template <int MP, int KPS>
+fg_status run_swap_t(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                     int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b, unsigned flags) {
+  constexpr int STAGES = swap_stages<MP, KPS>();
   fg::SwapParams p;
   // swap-AB: the MMA's A operand is the weight tile (B of the GEMM), its B operand the tokens
   p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_b), static_cast<uint32_t>(fmt_a));
@@ -550,14 +609,36 @@ fg_status run_swap(const Ctx* st, const void* A, const float* sfa, const void* B
   if (p.n_tiles > kCounterCapacity) return FG_ERR_UNSUPPORTED;
 
   CUtensorMap mW, mT;
-  if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
-  if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
-  const SwapChoice c = swap_choose<MP>(st->sms, p.n_tiles, p.num_kb);
+  if constexpr (KPS == 1) {
+    if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
+    if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
+  } else {
+    if (!encode_fp8_map_kblocks(&mW, B, K, N, kBlockM, KPS)) return FG_ERR_CUDA;
+    if (!encode_fp8_map_kblocks(&mT, A, K, M, MP, KPS)) return FG_ERR_CUDA;
+  }
+  const SwapChoice c = swap_choose<MP, KPS>(st->sms, p.n_tiles, p.num_kb);
   p.tile_aligned = c.tile_aligned;
   p.cluster = c.cluster;
   void* args[3] = {&mW, &mT, &p};
-  return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(c.grid), swap_smem_bytes<MP, STAGES>(), stream,
-                                                               args, fg::kThreads, 0, c.cluster);
+  return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES, KPS>>(
+      dim3(c.grid), swap_smem_bytes<MP, STAGES, KPS>(), stream, args, fg::kThreads, 0, c.cluster);
+}
+
+// K blocks per stage for a small-M call: 2 when K is a multiple of 128 (the 3-D copies need whole
+// K blocks) and has at least 4 of them (so that a tile still splits into two or more units for the
+// cluster and stream-K schedules), unless fg_set_swap_kps says otherwise (2: whenever K allows).
+int swap_kps_for(int K) {
+  const int f = g_swap_kps.load(std::memory_order_relaxed);
+  if (K % kBlockK != 0 || f == 1) return 1;
+  return (f == 2 || K / kBlockK >= 4) ? 2 : 1;
+}
+
+template <int MP>
+fg_status run_swap(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
+                   int M, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b, unsigned flags) {
+  if (swap_kps_for(K) == 2)
+    return run_swap_t<MP, 2>(st, A, sfa, B, sfb, C, M, N, K, stream, fmt_a, fmt_b, flags);
+  return run_swap_t<MP, 1>(st, A, sfa, B, sfb, C, M, N, K, stream, fmt_a, fmt_b, flags);
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -713,6 +794,17 @@ uint64_t fg_launch_count(void) { return g_launches.load(); }
 
 int fg_debug_set_stall(int enable) { return g_debug_stall.exchange(enable ? 1 : 0); }
 
+int fg_tile_plan(int layout, int M, int N, int K, int G) {
+  if (layout < 0 || layout > 2 || M <= 0 || N <= 0 || K <= 0 || G <= 0) return -1;
+  fg_status err;
+  const DeviceState* st = state_for_current(&err);
+  if (!st) return -1;
+  const int path = g_dense_path.load();
+  if (layout == 0 && (path == 2 || (path == 0 && M <= kMaxSwapMP))) return 2000;
+  const TilePlan t = tile_plan(layout, M, N, G, st->sms);
+  return t.kernel * 1000 + t.bn;
+}
+
 int fg_set_tile_n(int bn) {
   if (bn != 0 && bn != 128 && bn != 192 && bn != 256) return g_tile_n.load();
   return g_tile_n.exchange(bn);
@@ -727,9 +819,19 @@ int fg_swap_plan(int M, int N, int K) {
   if (!st) return -1;
   const int tiles = (N + kBlockM - 1) / kBlockM;
   const int kb = (K + kBlockK - 1) / kBlockK;
-  const SwapChoice c = M <= 32 ? swap_choose<32>(st->sms, tiles, kb)
-                       : M <= 64 ? swap_choose<64>(st->sms, tiles, kb) : swap_choose<128>(st->sms, tiles, kb);
+  SwapChoice c;
+  if (swap_kps_for(K) == 2)
+    c = M <= 32 ? swap_choose<32, 2>(st->sms, tiles, kb)
+                : M <= 64 ? swap_choose<64, 2>(st->sms, tiles, kb) : swap_choose<128, 2>(st->sms, tiles, kb);
+  else
+    c = M <= 32 ? swap_choose<32, 1>(st->sms, tiles, kb)
+                : M <= 64 ? swap_choose<64, 1>(st->sms, tiles, kb) : swap_choose<128, 1>(st->sms, tiles, kb);
   return c.cluster > 1 ? c.cluster : c.tile_aligned;
+}
+
+int fg_set_swap_kps(int kps) {
+  if (kps != 0 && kps != 1 && kps != 2) return g_swap_kps.load();
+  return g_swap_kps.exchange(kps);
 }
 
 int fg_set_swap_schedule(int schedule) {
@@ -785,7 +887,6 @@ fg_status fp8_gemm_nt_ws(const void* A, const float* sfa, const void* B, const f
     if (M <= 64) return run_swap<64>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b, flags);
     return run_swap<128>(st, A, sfa, B, sfb, C, M, N, K, cs, fmt_a, fmt_b, flags);
   }
-  if (path == 3) return dispatch_pair<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
   return dispatch_tiled<fg::kDense>(st, A, sfa, B, sfb, C, nullptr, nullptr, M, 1, N, K, cs, fmt_a, fmt_b);
 }
 
@@ -848,9 +949,6 @@ fg_status fp8_gemm_grouped_masked_ws(const void* A, const float* sfa, const void
   Ctx ctx;
   s = resolve_ctx(workspace, workspace_bytes, &ctx);
   if (s != FG_OK) return s;
-  if (g_dense_path.load() == 3)
-    return dispatch_pair<fg::kMasked>(&ctx, A, sfa, B, sfb, C, masked_m, Mmax, G, N, K,
-                                      static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
   return dispatch_tiled<fg::kMasked>(&ctx, A, sfa, B, sfb, C, nullptr, masked_m, Mmax, G, N, K,
                                 static_cast<cudaStream_t>(stream), fmt_a, fmt_b);
 }

@@ -92,6 +92,31 @@ def test_tile_widths(fg, bn, M, N, K):
         fg.set_tiled_streamk(old_sk)
 
 
+@pytest.mark.parametrize("schedule", [0, -1, 1, 2, 4, 8])
+@pytest.mark.parametrize("M,N,K", [(64, 2112, 7168), (128, 7168, 2048), (32, 1032, 1408), (100, 4096, 640),
+                                   (7, 264, 384)])
+def test_swap_two_kblocks_per_stage(fg, schedule, M, N, K):
+    """The small-M kernel with two K blocks per ring stage (3-D copies; the default when K is a
+    multiple of 128) against the oracle on every schedule, odd K-block counts included (the last
+    stage of a tile then holds one K block); with whole tiles, bit-identical to one K block per
+    stage (the same fp32 operations in the same order)."""
+    case = synth.dense_case(800 + M, M, N, K, row_scaled=True)
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
+    old = fg.set_swap_schedule(schedule)
+    try:
+        fg.set_swap_kps(2)
+        two = run_dense(fg, case, 2)
+        fg.set_swap_kps(1)
+        one = run_dense(fg, case, 2)
+    finally:
+        fg.set_swap_kps(0)
+        fg.set_swap_schedule(old)
+    close(two, ref, f"kps=2 {M}x{N}x{K} schedule {schedule}")
+    close(one, ref, f"kps=1 {M}x{N}x{K} schedule {schedule}")
+    if schedule == 1:
+        np.testing.assert_array_equal(two, one)
+
+
 @pytest.mark.parametrize("w", workloads.decode_sweep(), ids=lambda w: w["name"])
 def test_decode_sweep_full(fg, w):
     case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"], row_scaled=True)
