@@ -543,7 +543,11 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local, static_b=Fal
     fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
     shapes = []
     sum_bytes_dom, sum_ms_dom, sum_ms_all = 0.0, 0.0, 0.0
-    dom = kernel_name(cases[0])
+    # the dominant kernel: the one with the largest share of the event-timed launch durations
+    share = {}
+    for c, ts in zip(cases, per_case_ms):
+        share[kernel_name(c)] = share.get(kernel_name(c), 0.0) + statistics.mean(ts)
+    dom = max(share, key=share.get)
     for c, w, wk, ts in zip(cases, wl, works, per_case_ms):
         ms = statistics.mean(ts)
         tfl = wk[0] / (ms * 1e-3) / 1e12
@@ -617,8 +621,8 @@ def run_ours(args, rank, world, local):
         fg.set_swap_schedule(args.swap_schedule)
     if args.tile_n is not None:
         fg.set_tile_n(args.tile_n)
-    if args.swap_kps is not None:
-        fg.set_swap_kps(args.swap_kps)
+    if args.stage_kblocks is not None:
+        fg.set_stage_kblocks(args.stage_kblocks)
     stream = torch.cuda.Stream(device=dev)
     name, wl = workload_list(args.workload, args.shape)
     # The weights of a decode step are loaded once and never rewritten, so the dense calls declare
@@ -673,7 +677,7 @@ def run_ours(args, rank, world, local):
                            tiled_streamk="library default" if args.tiled_streamk is None else args.tiled_streamk,
                            swap_schedule="library default" if args.swap_schedule is None else args.swap_schedule,
                            tile_n="library default" if args.tile_n is None else args.tile_n,
-                           swap_kps="library default" if args.swap_kps is None else args.swap_kps),
+                           stage_kblocks="library default" if args.stage_kblocks is None else args.stage_kblocks),
             "hbm_gbs": res["hbm_gbs"], "shapes": res["shapes"], "shapes_timing": res["shapes_timing"],
             "roofline": res["roofline"],
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
@@ -733,8 +737,9 @@ def main():
                          "cluster split, 1 whole tiles, 2/4/8 the cluster split with that many CTAs per tile")
     ap.add_argument("--tile-n", type=int, default=None, choices=[0, 128, 192, 256],
                     help="output tile width of the tiled / CTA-pair kernels (fg_set_tile_n): 0 automatic")
-    ap.add_argument("--swap-kps", type=int, default=None, choices=[0, 1, 2],
-                    help="K blocks per ring stage of the small-M kernel (fg_set_swap_kps): 0 automatic")
+    ap.add_argument("--stage-kblocks", type=int, default=None, choices=[0, 1, 2],
+                    help="K blocks per ring stage of the small-M and CTA-pair kernels (fg_set_stage_kblocks): "
+                         "0 automatic")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

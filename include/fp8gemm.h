@@ -289,14 +289,14 @@ int fg_set_tiled_streamk(int overhead);
  * order.  Returns the previous value. */
 int fg_set_swap_schedule(int schedule);
 
-/* K blocks per ring stage of the small-M kernel, process-wide: 0 (default) = automatic -- 2
- * when K is a multiple of 128 with at least four K blocks, each weight and token copy then
- * moving two K blocks at once (a CTA's copy rate is bounded by the number of copies in flight
- * more than by their size) -- else 1; 1 forces single K blocks; 2 forces pairs wherever K is a
- * multiple of 128.  Any other value is ignored.  Results agree to fp32 summation order (split
- * points of the K range move to pair boundaries).
- * Returns the previous value. */
-int fg_set_swap_kps(int kps);
+/* K blocks per ring stage of the small-M (swap-AB) and CTA-pair kernels, process-wide.
+ * 0 (default) = automatic: 2 when K is a multiple of 128 (the small-M kernel also needs at
+ * least four K blocks), each operand copy then moving two K blocks at once -- a CTA's copy
+ * rate is bounded by the number of copies in flight more than by their size -- else 1.
+ * 1 forces single K blocks; 2 forces pairs wherever K is a multiple of 128.  Any other value
+ * is ignored.  Results agree to fp32 summation order (split points of the small-M kernel's
+ * K range move to pair boundaries).  Returns the previous value. */
+int fg_set_stage_kblocks(int kps);
 
 /* The schedule the small-M kernel takes for a dense call of this shape on the current
  * device under the current setting: S (2, 4 or 8) for the cluster split, 1 for whole

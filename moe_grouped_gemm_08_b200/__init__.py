@@ -78,8 +78,8 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_set_tile_n.restype = _int
     l.fg_set_tiled_streamk.argtypes = [_int]
     l.fg_set_tiled_streamk.restype = _int
-    l.fg_set_swap_kps.argtypes = [_int]
-    l.fg_set_swap_kps.restype = _int
+    l.fg_set_stage_kblocks.argtypes = [_int]
+    l.fg_set_stage_kblocks.restype = _int
     l.fg_set_swap_schedule.argtypes = [_int]
     l.fg_set_swap_schedule.restype = _int
     l.fg_swap_plan.argtypes = [_int, _int, _int]
@@ -182,10 +182,10 @@ def set_swap_schedule(schedule: int) -> int:
     return int(_lib.fg_set_swap_schedule(int(schedule)))
 
 
-def set_swap_kps(kps: int) -> int:
-    """K blocks per ring stage of the small-M kernel: 0 automatic (2 when K % 128 == 0), 1 or 2.
-    Returns the old value."""
-    return int(_lib.fg_set_swap_kps(int(kps)))
+def set_stage_kblocks(kps: int) -> int:
+    """K blocks per ring stage of the small-M and CTA-pair kernels: 0 automatic (2 when K % 128 == 0),
+    1 or 2. Returns the old value."""
+    return int(_lib.fg_set_stage_kblocks(int(kps)))
 
 
 def swap_plan(M: int, N: int, K: int) -> int:

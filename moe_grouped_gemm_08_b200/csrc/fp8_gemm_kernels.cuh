@@ -832,7 +832,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 // tempty[b] of the leader counts the promotion warps of both CTAs.  Cluster barriers only right
 // after set-up and right before teardown, which every thread of both CTAs reaches; every other
 // wait is bounded.
-template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0)>
+// KPS: K blocks per ring stage.  KPS > 1 (K a multiple of 128) loads KPS consecutive K blocks of
+// each operand with one 4-D copy over {128 bytes, rows, K blocks, groups}, laid out as KPS tiles
+// one after the other (as KPS 3-D copies would), halving the copies per byte.
+template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0), int KPS = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
@@ -841,9 +844,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
   constexpr int NCH = COLS / 32;  // 32-column TMEM loads (and store boxes) per thread
   static_assert(COLS % 32 == 0 && BN <= 256, "BN");
   constexpr int PAIR_ROWS = 2 * kBlockM;
-  constexpr int A_BYTES = kBlockM * kBlockK;   // this CTA's 128 rows of A
-  constexpr int B_BYTES = COLS * kBlockK;      // this CTA's half of the B tile
-  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int A_BYTES = kBlockM * kBlockK;   // one K block of this CTA's 128 rows of A
+  constexpr int B_BYTES = COLS * kBlockK;      // one K block of this CTA's half of the B tile
+  constexpr int STAGE_BYTES = KPS * (A_BYTES + B_BYTES);  // [KPS A tiles][KPS B tiles]
   constexpr int NUM_TBUF = 512 / BN;
   constexpr uint32_t TMEM_COLS = 512;
   constexpr int CHUNK_FLOATS = kSaChunk * kBlockM + 2 * kSaChunk;
@@ -942,12 +945,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
         const int a_row = ti.m0 + static_cast<int>(rank) * kBlockM;
         const int b_row = ti.n0 + static_cast<int>(rank) * COLS;
         FG_DCHECK(ti.m0 >= 0 && ti.m0 < p.M && ti.n0 >= 0 && ti.n0 < p.N && ti.g >= 0 && ti.g < p.G, p.status);
-        for (int kb = 0; kb < p.num_kb; ++kb) {
+        for (int kb = 0; kb < p.num_kb; kb += KPS) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
           uint8_t* st = smem + stage * STAGE_BYTES;
           if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-          tma_load_3d_pair(st, &tmA, full_leader + stage * 8, kb * kBlockK, a_row, ga, pol_a);
-          tma_load_3d_pair(st + A_BYTES, &tmB, full_leader + stage * 8, kb * kBlockK, b_row, gb, pol_b);
+          if constexpr (KPS == 1) {
+            tma_load_3d_pair(st, &tmA, full_leader + stage * 8, kb * kBlockK, a_row, ga, pol_a);
+            tma_load_3d_pair(st + A_BYTES, &tmB, full_leader + stage * 8, kb * kBlockK, b_row, gb, pol_b);
+          } else {
+            tma_load_4d_pair(st, &tmA, full_leader + stage * 8, 0, a_row, kb, ga, pol_a);
+            tma_load_4d_pair(st + KPS * A_BYTES, &tmB, full_leader + stage * 8, 0, b_row, kb, gb, pol_b);
+          }
           ++issued;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -969,21 +977,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
         uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
         bool ok = true;
         for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-          for (int kb = 0; kb < p.num_kb; ++kb) {
+          for (int kb = 0; kb < p.num_kb && ok; kb += KPS) {
             if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) { ok = false; break; }
-            if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t d = tmem_base + tb * BN;
-            const uint32_t st = smem_addr(smem + stage * STAGE_BYTES);
-            const uint64_t adesc = smem_desc_k128_sw128(st);
-            const uint64_t bdesc = smem_desc_k128_sw128(st + A_BYTES);
+            const int nk = (p.num_kb - kb) < KPS ? (p.num_kb - kb) : KPS;
+            for (int i = 0; i < nk; ++i) {
+              if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
+              tc_fence_after();
+              const uint32_t d = tmem_base + tb * BN;
+              const uint32_t st = smem_addr(smem + stage * STAGE_BYTES);
+              const uint64_t adesc = smem_desc_k128_sw128(st + i * A_BYTES);
+              const uint64_t bdesc = smem_desc_k128_sw128(st + KPS * A_BYTES + i * B_BYTES);
 #pragma unroll
-            for (int j = 0; j < kBlockK / 32; ++j)
-              mma_f8_pair(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
-            mma_commit_pair(&empty[stage], kBoth);
-            mma_commit_pair(&tfull[tb], kBoth);
+              for (int j = 0; j < kBlockK / 32; ++j)
+                mma_f8_pair(d, adesc + 2 * j, bdesc + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
+              if (i == nk - 1) mma_commit_pair(&empty[stage], kBoth);
+              mma_commit_pair(&tfull[tb], kBoth);
+              if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
+            }
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            if (++tb == NUM_TBUF) { tb = 0; tphase ^= 1u; }
           }
         }
         mma_commit_pair(mma_done, kBoth);  // arrives on both CTAs once every pair MMA has finished

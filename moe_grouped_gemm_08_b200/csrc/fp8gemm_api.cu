@@ -87,9 +87,9 @@ template <int BN>
 constexpr int tiled_stages() {
   return BN == 128 ? 5 : (BN == 192 ? kTiledStages : 3);
 }
-template <int BN>
+template <int BN, int KPS = 1>
 constexpr int pair_stages() {
-  return BN == 192 ? kPairStages : 4;
+  return KPS == 1 ? (BN == 192 ? kPairStages : 4) : 2;
 }
 
 template <int BN, int STAGES>
@@ -103,14 +103,16 @@ static_assert(tiled_smem_bytes<kTiledBN, kTiledStages>() <= 227 * 1024, "tiled k
 static_assert(tiled_smem_bytes<128, tiled_stages<128>()>() <= 227 * 1024, "tiled kernel shared memory");
 static_assert(tiled_smem_bytes<256, tiled_stages<256>()>() <= 227 * 1024, "tiled kernel shared memory");
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int KPS = 1>
 constexpr size_t pair_smem_bytes() {
-  return 1024 + static_cast<size_t>(STAGES) * (kBlockM + BN / 2) * kBlockK +
+  return 1024 + static_cast<size_t>(STAGES) * KPS * (kBlockM + BN / 2) * kBlockK +
          static_cast<size_t>(fg::kPromoWarps) * (BN / 64) * fg::kStoreBoxBytes +
          2 * (fg::kSaChunk * kBlockM + 2 * fg::kSaChunk) * 4 + 256 + 4 * (fg::kMaskedMaxGroups + 1);
 }
 static_assert(pair_smem_bytes<kPairBN, kPairStages>() <= 227 * 1024, "pair kernel shared memory");
 static_assert(pair_smem_bytes<256, pair_stages<256>()>() <= 227 * 1024, "pair kernel shared memory");
+static_assert(pair_smem_bytes<256, pair_stages<256, 2>(), 2>() <= 227 * 1024, "pair kernel shared memory");
+static_assert(pair_smem_bytes<192, pair_stages<192, 2>(), 2>() <= 227 * 1024, "pair kernel shared memory");
 
 // Ring stages of the small-M kernel by MP and K blocks per stage (KPS): about 192 KB of ring.
 template <int MP, int KPS = 1>
@@ -128,8 +130,15 @@ static_assert(swap_smem_bytes<64, swap_stages<64, 2>(), 2>() <= 227 * 1024, "swa
 static_assert(swap_smem_bytes<128, swap_stages<128, 2>(), 2>() <= 227 * 1024, "swap kernel shared memory");
 
 // K blocks per stage of the small-M kernel: 0 automatic (2 when K is a multiple of 128, else 1),
-// or 1 / 2 forced (2 only where K allows it; fg_set_swap_kps)
-std::atomic<int> g_swap_kps{0};
+// or 1 / 2 forced (2 only where K allows it; fg_set_stage_kblocks)
+std::atomic<int> g_stage_kb{0};
+
+// K blocks per stage of the CTA-pair kernel: 2 when K is a multiple of 128 with at least two K
+// blocks, unless fg_set_stage_kblocks forces 1.
+int pair_kps_for(int K) {
+  const int f = g_stage_kb.load(std::memory_order_relaxed);
+  return (K % 128 == 0 && K >= 256 && f != 1) ? 2 : 1;
+}
 
 int current_device() {
   int dev = -1;
@@ -212,6 +221,21 @@ bool encode_fp8_map_kblocks(CUtensorMap* map, const void* base, uint64_t K, uint
   cuuint32_t box[3] = {static_cast<cuuint32_t>(kBlockK), box_rows, kps};
   cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 4-D view of a grouped K-major e4m3 tensor [groups, rows, K] (K a multiple of 128) as {128 bytes,
+// rows, K blocks, groups}: a box {128, box_rows, kps, 1} is kps consecutive K blocks of box_rows
+// rows of one group, laid out as kps swizzled tiles one after the other.
+bool encode_fp8_map_kblocks_grouped(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint64_t groups,
+                                    uint32_t box_rows, uint32_t kps) {
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(kBlockK), rows, K / kBlockK, groups};
+  cuuint64_t strides[3] = {K, static_cast<cuuint64_t>(kBlockK), K * rows};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(kBlockK), box_rows, kps, 1};
+  cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estride,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -378,12 +402,13 @@ int pair_capacity(int sms, size_t smem) {
   return n;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int KPS = 1>
 fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
-  constexpr int STAGES = pair_stages<BN>();
-  constexpr auto KERNEL = fg::fp8_gemm_pair_kernel<BN, STAGES, MODE>;
-  constexpr size_t SMEM = pair_smem_bytes<BN, STAGES>();
+  constexpr int STAGES = pair_stages<BN, KPS>();
+  constexpr auto KERNEL =
+      fg::fp8_gemm_pair_kernel<BN, STAGES, MODE, (BN > 192 ? FG_PIPE_256 : 0), KPS>;
+  constexpr size_t SMEM = pair_smem_bytes<BN, STAGES, KPS>();
   fg::TiledParams p;
   p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
   p.ws = nullptr;
@@ -417,8 +442,13 @@ fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B
   CUtensorMap mA, mB, mC;
   const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;
   const uint64_t groupsB = (MODE == fg::kDense) ? 1 : static_cast<uint64_t>(G);
-  if (!encode_fp8_map(&mA, A, K, M, groupsA, kBlockM)) return FG_ERR_CUDA;
-  if (!encode_fp8_map(&mB, B, K, N, groupsB, BN / 2)) return FG_ERR_CUDA;
+  if constexpr (KPS == 1) {
+    if (!encode_fp8_map(&mA, A, K, M, groupsA, kBlockM)) return FG_ERR_CUDA;
+    if (!encode_fp8_map(&mB, B, K, N, groupsB, BN / 2)) return FG_ERR_CUDA;
+  } else {
+    if (!encode_fp8_map_kblocks_grouped(&mA, A, K, M, groupsA, kBlockM, KPS)) return FG_ERR_CUDA;
+    if (!encode_fp8_map_kblocks_grouped(&mB, B, K, N, groupsB, BN / 2, KPS)) return FG_ERR_CUDA;
+  }
   if (!encode_bf16_store_map(&mC, C, N, M, groupsA, MODE == fg::kMasked)) return FG_ERR_CUDA;
 
   const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
@@ -470,11 +500,13 @@ fg_status dispatch_tiled(const Ctx* st, const void* A, const float* sfa, const v
                          int fmt_a, int fmt_b) {
   const TilePlan t = tile_plan(MODE, M, N, G, st->sms);
   if (t.kernel == 3 && MODE != fg::kContiguous) {
+    constexpr int PM = MODE == fg::kContiguous ? fg::kDense : MODE;  // (never the contiguous layout)
+    const bool pairs = pair_kps_for(K) == 2;
     if (t.bn == 256)
-      return run_pair<MODE == fg::kContiguous ? fg::kDense : MODE, 256>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K,
-                                                                         stream, fmt_a, fmt_b);
-    return run_pair<MODE == fg::kContiguous ? fg::kDense : MODE, kPairBN>(st, A, sfa, B, sfb, C, masked_m, M, G, N,
-                                                                            K, stream, fmt_a, fmt_b);
+      return pairs ? run_pair<PM, 256, 2>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b)
+                   : run_pair<PM, 256, 1>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
+    return pairs ? run_pair<PM, kPairBN, 2>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b)
+                 : run_pair<PM, kPairBN, 1>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
   }
   if (t.bn == 128)
     return run_tiled<MODE, 128>(st, A, sfa, B, sfb, C, m_indices, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
@@ -626,9 +658,9 @@ fg_status run_swap_t(const Ctx* st, const void* A, const float* sfa, const void*
 
 // K blocks per stage for a small-M call: 2 when K is a multiple of 128 (the 3-D copies need whole
 // K blocks) and has at least 4 of them (so that a tile still splits into two or more units for the
-// cluster and stream-K schedules), unless fg_set_swap_kps says otherwise (2: whenever K allows).
+// cluster and stream-K schedules), unless fg_set_stage_kblocks says otherwise (2: whenever K allows).
 int swap_kps_for(int K) {
-  const int f = g_swap_kps.load(std::memory_order_relaxed);
+  const int f = g_stage_kb.load(std::memory_order_relaxed);
   if (K % kBlockK != 0 || f == 1) return 1;
   return (f == 2 || K / kBlockK >= 4) ? 2 : 1;
 }
@@ -829,9 +861,9 @@ int fg_swap_plan(int M, int N, int K) {
   return c.cluster > 1 ? c.cluster : c.tile_aligned;
 }
 
-int fg_set_swap_kps(int kps) {
-  if (kps != 0 && kps != 1 && kps != 2) return g_swap_kps.load();
-  return g_swap_kps.exchange(kps);
+int fg_set_stage_kblocks(int kps) {
+  if (kps != 0 && kps != 1 && kps != 2) return g_stage_kb.load();
+  return g_stage_kb.exchange(kps);
 }
 
 int fg_set_swap_schedule(int schedule) {

@@ -104,12 +104,12 @@ def test_swap_two_kblocks_per_stage(fg, schedule, M, N, K):
     ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"])
     old = fg.set_swap_schedule(schedule)
     try:
-        fg.set_swap_kps(2)
+        fg.set_stage_kblocks(2)
         two = run_dense(fg, case, 2)
-        fg.set_swap_kps(1)
+        fg.set_stage_kblocks(1)
         one = run_dense(fg, case, 2)
     finally:
-        fg.set_swap_kps(0)
+        fg.set_stage_kblocks(0)
         fg.set_swap_schedule(old)
     close(two, ref, f"kps=2 {M}x{N}x{K} schedule {schedule}")
     close(one, ref, f"kps=1 {M}x{N}x{K} schedule {schedule}")
