@@ -254,6 +254,12 @@ int fg_set_dense_path(int path);
  * Returns the previous value. */
 int fg_set_tile_n(int bn);
 
+/* Promotion warpgroups of the 256-wide CTA-pair kernel, process-wide: 2 (default) or 4.  With
+ * 4 (640 threads per CTA), each SM sub-partition runs four promotion warps, each holding a
+ * quarter of its CTA's 128 x 256 accumulators.  Other values are ignored.  Results are
+ * identical.  Returns the previous value. */
+int fg_set_pair_promotion(int warpgroups);
+
 /* The kernel and tile width a call of this shape takes on the current device under the
  * current settings, as kernel * 1000 + width: 1xxx the one-CTA tiled kernel, 3xxx the
  * CTA pair, 2000 the small-M swap-AB kernel (dense, M <= 128).  layout: 0 dense, 1

@@ -72,6 +72,8 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_set_dense_path.restype = _int
     l.fg_debug_set_stall.argtypes = [_int]
     l.fg_debug_set_stall.restype = _int
+    l.fg_set_pair_promotion.argtypes = [_int]
+    l.fg_set_pair_promotion.restype = _int
     l.fg_tile_plan.argtypes = [_int, _int, _int, _int, _int]
     l.fg_tile_plan.restype = _int
     l.fg_set_tile_n.argtypes = [_int]
@@ -160,6 +162,11 @@ def set_tile_n(bn: int) -> int:
     """Output tile width of the tiled / CTA-pair kernels: 0 automatic, or 128, 192, 256. Returns the
     old value."""
     return int(_lib.fg_set_tile_n(int(bn)))
+
+
+def set_pair_promotion(warpgroups: int) -> int:
+    """Promotion warpgroups of the 256-wide CTA-pair kernel: 2 or 4. Returns the old value."""
+    return int(_lib.fg_set_pair_promotion(int(warpgroups)))
 
 
 def tile_plan(layout: str, M: int, N: int, K: int, G: int = 1) -> int:

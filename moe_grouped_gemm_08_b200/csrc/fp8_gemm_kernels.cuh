@@ -327,6 +327,7 @@ __device__ __forceinline__ void load_scale_chunk(const TiledParams& p, const Til
                                                  ScaleChunkRegs& r) {
   r.a = make_float4(0.f, 0.f, 0.f, 0.f);
   r.b = 0.0f;
+  if (tid >= kPromoWarps * 32) return;  // the first 256 promotion threads stage the scales
   const int kb = chunk * kSaChunk + (tid >> 5);
   const int r4 = (tid & 31) * 4;
   if (kb < p.num_kb) {
@@ -353,6 +354,7 @@ __device__ __forceinline__ void load_scale_chunk(const TiledParams& p, const Til
 
 // chunk layout in shared memory: sa[kSaChunk][128] floats, then sb[2][kSaChunk] floats
 __device__ __forceinline__ void store_scale_chunk(float* buf, int tid, const ScaleChunkRegs& r) {
+  if (tid >= kPromoWarps * 32) return;
   reinterpret_cast<float4*>(buf + (tid >> 5) * kBlockM + (tid & 31) * 4)[0] = r.a;
   if (tid < 2 * kSaChunk) buf[kSaChunk * kBlockM + tid] = r.b;
 }
@@ -819,6 +821,18 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
   if (threadIdx.x == 0 && *abort_flag) report_timeout(p.status);
 }
 
+// Thread shape of the CTA-pair kernel by promotion warpgroups PW: launch size, registers per
+// thread at launch (the compiler's cap for that size), and the setmaxnreg split between the PW
+// promotion warpgroups and the producer / MMA warpgroup.
+template <int PW>
+struct PairShape {
+  static constexpr int threads = (PW + 1) * 128;
+  static constexpr int launch_regs = PW == 2 ? kTiledLaunchRegs : 96;
+  static constexpr int promo_regs = PW == 2 ? 232 : 112;
+  static constexpr int ctrl_regs = PW == 2 ? 40 : 32;
+  static_assert(PW * 128 * promo_regs + 128 * ctrl_regs <= threads * launch_regs, "register split");
+};
+
 // ============================================================================
 // Kernel 3: CTA-pair tiled (dense M > 128, masked)
 // ============================================================================
@@ -835,17 +849,24 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
 // KPS: K blocks per ring stage.  KPS > 1 (K a multiple of 128) loads KPS consecutive K blocks of
 // each operand with one 4-D copy over {128 bytes, rows, K blocks, groups}, laid out as KPS tiles
 // one after the other (as KPS 3-D copies would), halving the copies per byte.
-template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0), int KPS = 1>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
+// PW: promotion warpgroups (2 or 4).  With 4, warpgroup h of the promotion warps owns columns
+// [h BN/4, (h+1) BN/4) of the tile, so every SM sub-partition runs four promotion warps instead of
+// two: twice the TMEM reads and FMAs in flight per K block, half the work per warp.
+template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0), int KPS = 1, int PW = 2>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<PW>::threads, 1)
     fp8_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
   static_assert(MODE != kContiguous, "a pair tile needs both 128-row halves in one group");
-  constexpr int COLS = BN / 2;    // columns per promotion thread
+  static_assert(PW == 2 || PW == 4, "PW");
+  constexpr int NPW = 4 * PW;                  // promotion warps
+  constexpr int PROD_WARP = NPW;               // TMA producer
+  constexpr int MMA_WARP = NPW + 1;            // TMEM owner + MMA issuer
+  constexpr int COLS = BN / PW;   // columns per promotion thread
   constexpr int NCH = COLS / 32;  // 32-column TMEM loads (and store boxes) per thread
   static_assert(COLS % 32 == 0 && BN <= 256, "BN");
   constexpr int PAIR_ROWS = 2 * kBlockM;
   constexpr int A_BYTES = kBlockM * kBlockK;   // one K block of this CTA's 128 rows of A
-  constexpr int B_BYTES = COLS * kBlockK;      // one K block of this CTA's half of the B tile
+  constexpr int B_BYTES = (BN / 2) * kBlockK;  // one K block of this CTA's half of the B tile
   constexpr int STAGE_BYTES = KPS * (A_BYTES + B_BYTES);  // [KPS A tiles][KPS B tiles]
   constexpr int NUM_TBUF = 512 / BN;
   constexpr uint32_t TMEM_COLS = 512;
@@ -857,7 +878,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_1024(smem_raw);  // same offsets in both CTAs: the pair MMA relies on it
   uint8_t* s_out = smem + STAGES * STAGE_BYTES;
-  float* s_scale = reinterpret_cast<float*>(s_out + kPromoWarps * WARP_STORE_BYTES);
+  float* s_scale = reinterpret_cast<float*>(s_out + NPW * WARP_STORE_BYTES);
   uint64_t* full = reinterpret_cast<uint64_t*>(s_scale + 2 * CHUNK_FLOATS);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
@@ -875,18 +896,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int num_pairs = static_cast<int>(gridDim.x >> 1);
 
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == PROD_WARP && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
     prefetch_tmap(&tmC);
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 2 * kPromoWarps); }
+    for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], 2 * NPW); }
     mbar_init(mma_done, 1);
-    mbar_init(pbar, kPromoWarps * 32);
+    mbar_init(pbar, NPW * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarp) { tmem_alloc_pair(tmem_slot, TMEM_COLS); tmem_relinquish_pair(); }
+  if (warp == MMA_WARP) { tmem_alloc_pair(tmem_slot, TMEM_COLS); tmem_relinquish_pair(); }
   tc_fence_before();
   __syncthreads();
   cluster_sync_all();  // both CTAs' barriers are initialised before either CTA signals the other
@@ -928,10 +949,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     num_tiles = p.m_blocks * p.n_blocks;  // m_blocks counts 256-row blocks here
   }
 
-  if (warp >= kPromoWarps) {
-    // ================================================ warpgroup 2: producer, MMA, idle warps
-    reg_dealloc<RegSplit<BN>::ctrl>();
-    if (warp == kProducerWarp && lane == 0) {
+  if (warp >= NPW) {
+    // ================================================ last warpgroup: producer, MMA, idle warps
+    reg_dealloc<PairShape<PW>::ctrl_regs>();
+    if (warp == PROD_WARP && lane == 0) {
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0;
       bool ok = true;
@@ -943,7 +964,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
         const int ga = (MODE == kMasked) ? ti.g : 0;
         const int gb = (MODE == kDense) ? 0 : ti.g;
         const int a_row = ti.m0 + static_cast<int>(rank) * kBlockM;
-        const int b_row = ti.n0 + static_cast<int>(rank) * COLS;
+        const int b_row = ti.n0 + static_cast<int>(rank) * (BN / 2);
         FG_DCHECK(ti.m0 >= 0 && ti.m0 < p.M && ti.n0 >= 0 && ti.n0 < p.N && ti.g >= 0 && ti.g < p.G, p.status);
         for (int kb = 0; kb < p.num_kb; kb += KPS) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
@@ -972,7 +993,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
           }
         }
       }
-    } else if (warp == kMmaWarp && lane == 0) {
+    } else if (warp == MMA_WARP && lane == 0) {
       if (leader) {
         uint32_t stage = 0, phase = 0, tb = 0, tphase = 0;
         bool ok = true;
@@ -1002,7 +1023,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     }
   } else {
     // ================================================ warpgroups 0-1: promotion + epilogue
-    reg_alloc<RegSplit<BN>::promo>();
+    reg_alloc<PairShape<PW>::promo_regs>();
     const int q = warp & 3;
     const int h = warp >> 2;
     const int row = q * 32 + lane;
@@ -1142,7 +1163,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == MMA_WARP) {
     // both CTAs: every pair MMA (which read this CTA's ring and wrote its TMEM) has finished; the
     // promotion above consumed every result, so this wait is short unless the CTA aborted
     if (lane == 0) {
@@ -1154,7 +1175,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kTiledThreads, 1)
     __syncwarp();
   }
   cluster_sync_all();  // neither CTA touches the other's barriers, ring or TMEM any more
-  if (warp == kMmaWarp) {
+  if (warp == MMA_WARP) {
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }

@@ -132,6 +132,8 @@ static_assert(swap_smem_bytes<128, swap_stages<128, 2>(), 2>() <= 227 * 1024, "s
 // K blocks per stage of the small-M kernel: 0 automatic (2 when K is a multiple of 128, else 1),
 // or 1 / 2 forced (2 only where K allows it; fg_set_stage_kblocks)
 std::atomic<int> g_stage_kb{0};
+// promotion warpgroups of the 256-wide CTA-pair kernel (2 or 4; fg_set_pair_promotion)
+std::atomic<int> g_pair_pw{2};
 
 // K blocks per stage of the CTA-pair kernel: 2 when K is a multiple of 128 with at least two K
 // blocks, unless fg_set_stage_kblocks forces 1.
@@ -376,7 +378,7 @@ fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* 
 // Largest number of CTA pairs of the pair kernel that can be resident at once (queried once per
 // device and kernel; clusters must fit inside a GPC, so this can be below #SMs / 2).
 template <auto KERNEL>
-int pair_capacity(int sms, size_t smem) {
+int pair_capacity(int sms, size_t smem, int threads) {
   static std::atomic<int> cached[kMaxDevices];
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return sms / 2;
@@ -391,7 +393,7 @@ int pair_capacity(int sms, size_t smem) {
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3(static_cast<unsigned>(sms & ~1), 1, 1);
-  cfg.blockDim = dim3(fg::kTiledThreads, 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
   cfg.dynamicSmemBytes = smem;
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, KERNEL, &cfg) != cudaSuccess || n <= 0) {
@@ -402,12 +404,13 @@ int pair_capacity(int sms, size_t smem) {
   return n;
 }
 
-template <int MODE, int BN, int KPS = 1>
+template <int MODE, int BN, int KPS = 1, int PW = 2>
 fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                    const int* masked_m, int M, int G, int N, int K, cudaStream_t stream, int fmt_a, int fmt_b) {
   constexpr int STAGES = pair_stages<BN, KPS>();
   constexpr auto KERNEL =
-      fg::fp8_gemm_pair_kernel<BN, STAGES, MODE, (BN > 192 ? FG_PIPE_256 : 0), KPS>;
+      fg::fp8_gemm_pair_kernel<BN, STAGES, MODE, (BN > 192 ? FG_PIPE_256 : 0), KPS, PW>;
+  using Shape = fg::PairShape<PW>;
   constexpr size_t SMEM = pair_smem_bytes<BN, STAGES, KPS>();
   fg::TiledParams p;
   p.fmt_bits = fg::idesc_formats(static_cast<uint32_t>(fmt_a), static_cast<uint32_t>(fmt_b));
@@ -452,11 +455,11 @@ fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B
   if (!encode_bf16_store_map(&mC, C, N, M, groupsA, MODE == fg::kMasked)) return FG_ERR_CUDA;
 
   const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks * (MODE == fg::kMasked ? G : 1);
-  const int cap = pair_capacity<KERNEL>(st->sms, SMEM);
+  const int cap = pair_capacity<KERNEL>(st->sms, SMEM, Shape::threads);
   const int pairs = static_cast<int>(tiles < cap ? tiles : cap);
   void* args[4] = {&mA, &mB, &mC, &p};
-  return launch<KERNEL>(dim3(static_cast<unsigned>(2 * pairs)), SMEM, stream, args, fg::kTiledThreads,
-                        fg::kTiledLaunchRegs);
+  return launch<KERNEL>(dim3(static_cast<unsigned>(2 * pairs)), SMEM, stream, args, Shape::threads,
+                        Shape::launch_regs);
 }
 
 // Kernel and output tile width of a call of the tiled family (dense M > 128, contiguous, masked).
@@ -502,6 +505,9 @@ fg_status dispatch_tiled(const Ctx* st, const void* A, const float* sfa, const v
   if (t.kernel == 3 && MODE != fg::kContiguous) {
     constexpr int PM = MODE == fg::kContiguous ? fg::kDense : MODE;  // (never the contiguous layout)
     const bool pairs = pair_kps_for(K) == 2;
+    if (t.bn == 256 && g_pair_pw.load(std::memory_order_relaxed) == 4)
+      return pairs ? run_pair<PM, 256, 2, 4>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b)
+                   : run_pair<PM, 256, 1, 4>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
     if (t.bn == 256)
       return pairs ? run_pair<PM, 256, 2>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b)
                    : run_pair<PM, 256, 1>(st, A, sfa, B, sfb, C, masked_m, M, G, N, K, stream, fmt_a, fmt_b);
@@ -859,6 +865,11 @@ int fg_swap_plan(int M, int N, int K) {
     c = M <= 32 ? swap_choose<32, 1>(st->sms, tiles, kb)
                 : M <= 64 ? swap_choose<64, 1>(st->sms, tiles, kb) : swap_choose<128, 1>(st->sms, tiles, kb);
   return c.cluster > 1 ? c.cluster : c.tile_aligned;
+}
+
+int fg_set_pair_promotion(int warpgroups) {
+  if (warpgroups != 2 && warpgroups != 4) return g_pair_pw.load();
+  return g_pair_pw.exchange(warpgroups);
 }
 
 int fg_set_stage_kblocks(int kps) {

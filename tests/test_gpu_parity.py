@@ -117,6 +117,26 @@ def test_swap_two_kblocks_per_stage(fg, schedule, M, N, K):
         np.testing.assert_array_equal(two, one)
 
 
+@pytest.mark.parametrize("pw", [2, 4])
+@pytest.mark.parametrize("M,N,K", [(300, 520, 1152), (513, 2048, 3072), (4096, 2112, 7168)])
+def test_pair_kernel_promotion_warpgroups(fg, pw, M, N, K):
+    """The 256-wide CTA-pair kernel with two and with four promotion warpgroups against the oracle
+    (sampled rows for the large shape); both give the same bits (identical arithmetic)."""
+    case = synth.dense_case(900 + M, M, N, K)
+    rows = sample_rows(M, 40, M) if M > 1024 else None
+    ref = oracle.gemm_nt(case["A"], case["sfa"], case["B"], case["sfb"], rows=rows)
+    old = (fg.set_tile_n(256), fg.set_pair_promotion(pw))
+    try:
+        got = run_dense(fg, case, 3)
+        fg.set_pair_promotion(2 if pw == 4 else 4)
+        other = run_dense(fg, case, 3)
+    finally:
+        fg.set_tile_n(old[0])
+        fg.set_pair_promotion(old[1])
+    close(got if rows is None else got[rows], ref, f"pair pw={pw} {M}x{N}x{K}")
+    np.testing.assert_array_equal(got, other)
+
+
 @pytest.mark.parametrize("w", workloads.decode_sweep(), ids=lambda w: w["name"])
 def test_decode_sweep_full(fg, w):
     case = synth.dense_case(w["seed"], w["M"], w["N"], w["K"], row_scaled=True)
