@@ -254,6 +254,28 @@ int fg_set_dense_path(int path);
  * Returns the previous value. */
 int fg_set_tile_n(int bn);
 
+/* Runtime specialisation of the one-CTA tiled kernel (the pages' library compiles its kernels at
+ * run time with the GEMM shape as constants: chattools.cn explainer, flashmla.org product page),
+ * process-wide, default 0 (off: the ahead-of-time kernels).  With 1, the first call of each
+ * shape that takes the one-CTA tiled kernel compiles it with NVRTC for sm_100a with that shape's
+ * K blocks, K, N, sfb blocks, tile columns and tile-walk grouping as compile-time constants, from
+ * the kernel sources embedded in this library, loads it and caches it (per device and shape);
+ * later calls launch it like the ahead-of-time kernel.  Compiling takes about two seconds, so
+ * make each shape's first call outside stream capture.  NVRTC (libnvrtc.so.12) and the CUDA
+ * headers are looked up at run time under $CUDA_HOME or /usr/local/cuda; without them the call
+ * returns FG_ERR_UNSUPPORTED (nothing falls back silently).  Results are bit-identical to the
+ * ahead-of-time kernel.  Returns the previous value. */
+int fg_set_jit(int enable);
+
+/* Number of runtime-specialised kernels compiled and cached in this process. */
+int fg_jit_cache_size(void);
+
+/* Compile (do not load) the runtime-specialised dense tiled kernel for tile width bn (128, 192,
+ * 256), num_kb K blocks of 128 and N columns; on success *cubin_bytes is the size of the sm_100a
+ * binary.  Needs NVRTC and the CUDA headers but no GPU.  FG_ERR_UNSUPPORTED without them,
+ * FG_ERR_CUDA if compilation fails, FG_ERR_INVALID_ARG for bad arguments. */
+fg_status fg_jit_compile_check(int bn, int num_kb, int N, size_t* cubin_bytes);
+
 /* Promotion warpgroups of the 256-wide CTA-pair kernel, process-wide: 2 (default) or 4.  With
  * 4 (640 threads per CTA), each SM sub-partition runs four promotion warps, each holding a
  * quarter of its CTA's 128 x 256 accumulators.  Other values are ignored.  Results are

@@ -72,6 +72,12 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_set_dense_path.restype = _int
     l.fg_debug_set_stall.argtypes = [_int]
     l.fg_debug_set_stall.restype = _int
+    l.fg_set_jit.argtypes = [_int]
+    l.fg_set_jit.restype = _int
+    l.fg_jit_cache_size.argtypes = []
+    l.fg_jit_cache_size.restype = _int
+    l.fg_jit_compile_check.argtypes = [_int, _int, _int, ctypes.POINTER(ctypes.c_size_t)]
+    l.fg_jit_compile_check.restype = _int
     l.fg_set_pair_promotion.argtypes = [_int]
     l.fg_set_pair_promotion.restype = _int
     l.fg_tile_plan.argtypes = [_int, _int, _int, _int, _int]
@@ -162,6 +168,22 @@ def set_tile_n(bn: int) -> int:
     """Output tile width of the tiled / CTA-pair kernels: 0 automatic, or 128, 192, 256. Returns the
     old value."""
     return int(_lib.fg_set_tile_n(int(bn)))
+
+
+def set_jit(enable: bool) -> int:
+    """Runtime specialisation of the one-CTA tiled kernel per shape (NVRTC). Returns the old value."""
+    return int(_lib.fg_set_jit(1 if enable else 0))
+
+
+def jit_cache_size() -> int:
+    return int(_lib.fg_jit_cache_size())
+
+
+def jit_compile_check(bn: int, num_kb: int, N: int) -> int:
+    """Compile the specialised dense tiled kernel (no GPU needed); returns the cubin size."""
+    n = ctypes.c_size_t(0)
+    _check(_lib.fg_jit_compile_check(int(bn), int(num_kb), int(N), ctypes.byref(n)), "fg_jit_compile_check")
+    return int(n.value)
 
 
 def set_pair_promotion(warpgroups: int) -> int:

@@ -34,7 +34,9 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#ifndef __CUDACC_RTC__
 #include <cstdint>
+#endif
 
 #include "sm100_ptx.cuh"
 
@@ -455,7 +457,20 @@ constexpr int kStoreBoxBytes = 32 * 64;
 template <int BN, int STAGES, int MODE, int PIPE = (BN > 192 ? FG_PIPE_256 : 0)>
 __global__ void __launch_bounds__(kTiledThreads, 1)
     fp8_gemm_tiled_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                          const __grid_constant__ CUtensorMap tmC, const TiledParams p) {
+                          const __grid_constant__ CUtensorMap tmC, const TiledParams p_in) {
+#ifdef FG_JIT_NUM_KB
+  // runtime-specialised build: the shape's K blocks, N, tile counts and tile-walk grouping are
+  // compile-time constants (the compiler unrolls and folds the walk arithmetic for this shape)
+  TiledParams p = p_in;
+  p.num_kb = FG_JIT_NUM_KB;
+  p.K = FG_JIT_K;
+  p.N = FG_JIT_N;
+  p.num_nb = FG_JIT_NUM_NB;
+  p.n_blocks = FG_JIT_N_BLOCKS;
+  p.group_m = FG_JIT_GROUP_M;
+#else
+  const TiledParams& p = p_in;
+#endif
   constexpr int COLS = BN / 2;  // columns per promotion thread
   constexpr int NCH = COLS / 32;  // 32-column TMEM loads (and store boxes) per thread
   // tiles start at multiples of 64 columns, so no 32-column chunk straddles a 128-column sfb block

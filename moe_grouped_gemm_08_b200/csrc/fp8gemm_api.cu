@@ -13,6 +13,8 @@
 #include "fp8_cast_kernels.cuh"
 #include "fp8_gemm_kernels.cuh"
 #include "fp8gemm.h"
+#include "fp8gemm_jit.h"
+#include "fg_jit_sources.inc"  // the kernel headers, embedded at build time (build.py)
 
 namespace {
 
@@ -315,6 +317,88 @@ fg_status check_common(const void* A, const float* sfa, const void* B, const flo
   return FG_OK;
 }
 
+// ------------------------------------------------------------------ runtime specialisation
+// fg_set_jit(1): the tiled kernel is compiled per shape with NVRTC (fp8gemm_jit.h) and cached.
+std::atomic<int> g_jit{0};
+std::mutex g_jit_mutex;
+// key: device, layout, tile width, stages, K blocks, K, N, sfb blocks, tile columns, grouping
+typedef std::tuple<int, int, int, int, int, int, int, int, int, int> JitKey;
+std::map<JitKey, CUfunction> g_jit_cache;
+
+// The -D constants and the name expression of one specialisation of the tiled kernel.
+std::vector<std::string> jit_defines(const fg::TiledParams& p) {
+  std::vector<std::string> d = {"FG_JIT_NUM_KB=" + std::to_string(p.num_kb), "FG_JIT_K=" + std::to_string(p.K),
+                                "FG_JIT_N=" + std::to_string(p.N), "FG_JIT_NUM_NB=" + std::to_string(p.num_nb),
+                                "FG_JIT_N_BLOCKS=" + std::to_string(p.n_blocks),
+                                "FG_JIT_GROUP_M=" + std::to_string(p.group_m),
+                                "FG_PIPE_256=" + std::to_string(FG_PIPE_256)};
+#ifdef FG_DEBUG
+  d.push_back("FG_DEBUG=1");
+#endif
+  return d;
+}
+std::string jit_name(int bn, int stages, int mode) {
+  const int pipe = bn > 192 ? FG_PIPE_256 : 0;
+  return "fg::fp8_gemm_tiled_kernel<" + std::to_string(bn) + ", " + std::to_string(stages) + ", " +
+         std::to_string(mode) + ", " + std::to_string(pipe) + ">";
+}
+
+// The specialised kernel for this call (compiled and loaded on first use), or nullptr with the
+// reason in *err: FG_ERR_UNSUPPORTED without NVRTC / CUDA headers, FG_ERR_CUDA if compiling,
+// loading or the register check failed.
+CUfunction jit_tiled_function(int mode, int bn, int stages, size_t smem, const fg::TiledParams& p, fg_status* err) {
+  std::lock_guard<std::mutex> lock(g_jit_mutex);
+  const JitKey key{current_device(), mode, bn, stages, p.num_kb, p.K, p.N, p.num_nb, p.n_blocks, p.group_m};
+  auto it = g_jit_cache.find(key);
+  if (it != g_jit_cache.end()) return it->second;
+  if (!fgjit::load_api() || !fgjit::load_driver()) {
+    *err = FG_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  std::vector<char> cubin;
+  std::string lowered, log;
+  const std::string name = jit_name(bn, stages, mode);
+  if (!fgjit::compile("#include \"fp8_gemm_kernels.cuh\"\n", kJitHeaderCount, kJitHeaderSources, kJitHeaderNames,
+                      name, jit_defines(p), &cubin, &lowered, &log)) {
+    *err = FG_ERR_CUDA;
+    return nullptr;
+  }
+  fgjit::Api& a = fgjit::api();
+  CUmodule mod;
+  CUfunction fn;
+  int regs = 0;
+  if (a.module_load(&mod, cubin.data()) != CUDA_SUCCESS || a.get_function(&fn, mod, lowered.c_str()) != CUDA_SUCCESS ||
+      a.get_attr(&regs, CU_FUNC_ATTRIBUTE_NUM_REGS, fn) != CUDA_SUCCESS || regs != fg::kTiledLaunchRegs ||
+      a.set_attr(fn, CU_FUNC_ATTRIBUTE_MAX_DYNAMIC_SHARED_SIZE_BYTES, static_cast<int>(smem)) != CUDA_SUCCESS) {
+    *err = FG_ERR_CUDA;
+    return nullptr;
+  }
+  g_jit_cache[key] = fn;
+  return fn;
+}
+
+// Launch a runtime-specialised kernel exactly as launch<>() launches the ahead-of-time one.
+fg_status jit_launch(CUfunction fn, dim3 grid, int threads, size_t smem, cudaStream_t stream, void** args) {
+  CUlaunchAttribute attr[1];
+  attr[0].id = CU_LAUNCH_ATTRIBUTE_PROGRAMMATIC_STREAM_SERIALIZATION;
+  attr[0].value.programmaticStreamSerializationAllowed = 1;
+  CUlaunchConfig cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDimX = grid.x;
+  cfg.gridDimY = grid.y;
+  cfg.gridDimZ = grid.z;
+  cfg.blockDimX = static_cast<unsigned>(threads);
+  cfg.blockDimY = 1;
+  cfg.blockDimZ = 1;
+  cfg.sharedMemBytes = static_cast<unsigned>(smem);
+  cfg.hStream = reinterpret_cast<CUstream>(stream);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (fgjit::api().launch(&cfg, fn, args, nullptr) != CUDA_SUCCESS) return FG_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return FG_OK;
+}
+
 template <int MODE, int BN>
 fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* B, const float* sfb, void* C,
                     const int* m_indices, const int* masked_m, int M, int G, int N, int K, cudaStream_t stream,
@@ -371,6 +455,12 @@ fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* 
       grid = static_cast<int>(ctas);
   }
   void* args[4] = {&mA, &mB, &mC, &p};
+  if (g_jit.load(std::memory_order_relaxed)) {
+    fg_status err = FG_OK;
+    CUfunction fn = jit_tiled_function(MODE, BN, STAGES, tiled_smem_bytes<BN, STAGES>(), p, &err);
+    if (!fn) return err;
+    return jit_launch(fn, dim3(grid), fg::kTiledThreads, tiled_smem_bytes<BN, STAGES>(), stream, args);
+  }
   return launch<fg::fp8_gemm_tiled_kernel<BN, STAGES, MODE>>(dim3(grid), tiled_smem_bytes<BN, STAGES>(), stream, args,
                                                               fg::kTiledThreads, fg::kTiledLaunchRegs);
 }
@@ -865,6 +955,35 @@ int fg_swap_plan(int M, int N, int K) {
     c = M <= 32 ? swap_choose<32, 1>(st->sms, tiles, kb)
                 : M <= 64 ? swap_choose<64, 1>(st->sms, tiles, kb) : swap_choose<128, 1>(st->sms, tiles, kb);
   return c.cluster > 1 ? c.cluster : c.tile_aligned;
+}
+
+int fg_set_jit(int enable) { return g_jit.exchange(enable ? 1 : 0); }
+
+int fg_jit_cache_size(void) {
+  std::lock_guard<std::mutex> lock(g_jit_mutex);
+  return static_cast<int>(g_jit_cache.size());
+}
+
+fg_status fg_jit_compile_check(int bn, int num_kb, int N, size_t* cubin_bytes) {
+  if (!cubin_bytes || num_kb <= 0 || N <= 0 || (bn != 128 && bn != 192 && bn != 256)) return FG_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_jit_mutex);
+  if (!fgjit::load_api()) return FG_ERR_UNSUPPORTED;
+  fg::TiledParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.num_kb = num_kb;
+  p.K = num_kb * kBlockK;
+  p.N = N;
+  p.num_nb = (N + kBlockK - 1) / kBlockK;
+  p.n_blocks = (N + bn - 1) / bn;
+  p.group_m = 1;
+  const int stages = bn == 128 ? tiled_stages<128>() : (bn == 192 ? tiled_stages<192>() : tiled_stages<256>());
+  std::vector<char> cubin;
+  std::string lowered, log;
+  if (!fgjit::compile("#include \"fp8_gemm_kernels.cuh\"\n", kJitHeaderCount, kJitHeaderSources, kJitHeaderNames,
+                      jit_name(bn, stages, fg::kDense), jit_defines(p), &cubin, &lowered, &log))
+    return FG_ERR_CUDA;
+  *cubin_bytes = cubin.size();
+  return FG_OK;
 }
 
 int fg_set_pair_promotion(int warpgroups) {

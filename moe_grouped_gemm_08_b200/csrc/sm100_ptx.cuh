@@ -4,8 +4,22 @@
 // hanging.  Nothing here is GEMM-specific.
 #pragma once
 
+#ifdef __CUDACC_RTC__
+// Runtime compilation (NVRTC, see fp8gemm_jit.cu): the fixed-width integer types and the opaque
+// 128-byte tensor-map type, without the host headers.
+typedef unsigned char uint8_t;
+typedef unsigned short uint16_t;
+typedef unsigned int uint32_t;
+typedef unsigned long long uint64_t;
+typedef int int32_t;
+typedef long long int64_t;
+typedef struct alignas(64) CUtensorMap_st {
+  unsigned long long opaque[16];
+} CUtensorMap;
+#else
 #include <cstdint>
 #include <cuda.h>
+#endif
 
 namespace fg {
 

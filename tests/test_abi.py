@@ -138,3 +138,13 @@ def test_workspace_entry_points_check_arguments_first():
     assert L.fp8_gemm_grouped_masked_ws(P16, P16, P16, P16, P16, P16, 2000, 64, 128, 128, 0, 0, 0, P16, 1 << 30,
                                         NULL) == 3
     assert L.fp8_gemm_nt_ws(P16, P16, P16, P16, P16, 0, 128, 128, 0, 0, 0, NULL, 0, NULL) == 0  # M = 0: no-op
+
+
+def test_runtime_specialisation_compiles_without_a_gpu():
+    """The runtime-specialisation path compiles the tiled kernel for sm_100a from the sources
+    embedded in the library (NVRTC; no GPU needed), for each tile width."""
+    for bn in (128, 192, 256):
+        assert fg.jit_compile_check(bn, 56, 4096) > 100_000
+    assert fg.lib.fg_jit_compile_check(100, 56, 4096, ctypes.byref(ctypes.c_size_t())) == 1  # bad width
+    old = fg.set_jit(True)
+    assert fg.set_jit(bool(old)) == 1
