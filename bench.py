@@ -606,6 +606,24 @@ def measure_workload(fg, name, wl, args, dev, stream, world, local, static_b=Fal
     return res, cases, devs, step_flops
 
 
+def box_copy_gbs(dev) -> float:
+    """This GPU's copy bandwidth now (read + write bytes of a 1 GiB bf16 copy, best of 5, CUDA events):
+    context for comparing runs on different machines; the roofline uses the measured peak."""
+    a = torch.empty(1 << 29, dtype=torch.bfloat16, device=dev)
+    b = torch.empty_like(a)
+    best = float("inf")
+    for _ in range(6):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        b.copy_(a)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    torch.cuda.empty_cache()
+    return round(2 * (1 << 30) / (best * 1e-3) / 1e9, 1)
+
+
 def run_ours(args, rank, world, local):
     import moe_grouped_gemm_08_b200 as fg
 
@@ -624,6 +642,7 @@ def run_ours(args, rank, world, local):
     if args.stage_kblocks is not None:
         fg.set_stage_kblocks(args.stage_kblocks)
     stream = torch.cuda.Stream(device=dev)
+    copy_gbs = box_copy_gbs(dev)
     name, wl = workload_list(args.workload, args.shape)
     # The weights of a decode step are loaded once and never rewritten, so the dense calls declare
     # them static (FG_FLAG_STATIC_B: weight tiles may load before the preceding launch ends);
@@ -682,7 +701,8 @@ def run_ours(args, rank, world, local):
             "roofline": res["roofline"],
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": res["gpu_launches"], "clocks": res["clocks"], "device_status": res["device_status"]}
+            "gpu_launches": res["gpu_launches"], "clocks": res["clocks"], "device_status": res["device_status"],
+            "box_copy_gbs": copy_gbs}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         s, f, cores = time_oracle(cases, row_fraction=1.0)
         line["cpu_baseline"] = {"value": round(f / s / 1e12, 5), "unit": "TFLOPS", "cores": cores, "kind": "oracle",
