@@ -1248,7 +1248,7 @@ __device__ __forceinline__ void cluster_reduce_store(const SwapParams& p, uint32
 template <int MP, int STAGES, int KPS = 1>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_swap_streamk_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmT,
-                                 const SwapParams p) {
+                                 const __grid_constant__ CUtensorMap tmC, const SwapParams p) {
   static_assert(MP == 32 || MP == 64 || MP == 128, "MP");
   static_assert(KPS == 1 || KPS == 2 || KPS == 4, "KPS");
   constexpr int W_BYTES = kBlockM * kBlockK;  // one K block of 128 weight rows
@@ -1335,6 +1335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmW);
     prefetch_tmap(&tmT);
+    prefetch_tmap(&tmC);
     for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int b = 0; b < NUM_TBUF; ++b) { mbar_init(&tfull[b], 1); mbar_init(&tempty[b], kPromoWarps); }
     mbar_init(mma_done, 1);
@@ -1421,21 +1422,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool first_segment = true;
     int chunk_base = u_begin, chunk_end = u_begin;  // units whose scales are staged
 
-    // bf16 tile from registers (thread = weight row nl, columns = tokens) -> C[m, t*128 + nl],
-    // transposed through shared memory so that the global stores are 16-byte row segments
+    // bf16 tile from registers (thread = weight row nl, columns = tokens) -> C[m, t*128 + nl]:
+    // transposed into the [token][weight row] staging tile, which one TMA store writes to C (rows
+    // past M and columns past N clipped by the tensor map).  The store runs on while the warps go on
+    // to the next tile; the staging tile is rewritten only after the store has read it.
+    bool store_pending = false;
     auto store_tile = [&](const float* vals, int n_base) -> bool {
+      if (store_pending) {
+        if (tid == 0) bulk_wait_read_all();
+        if (!group_sync(pbar, pphase, abort_flag)) return false;
+      }
 #pragma unroll
       for (int j = 0; j < COLS; ++j) s_c[(h * COLS + j) * kBlockM + nl] = __float2bfloat16_rn(vals[j]);
+      fence_proxy_async_smem();
       if (!group_sync(pbar, pphase, abort_flag)) return false;
-      const int rows = p.M < MP ? p.M : MP;
-      for (int i = tid; i < rows * (kBlockM / 8); i += NPROMO) {
-        const int mm = i / (kBlockM / 8), ch = i % (kBlockM / 8);
-        if (n_base + ch * 8 < p.N) {
-          const uint4 val = *reinterpret_cast<const uint4*>(s_c + mm * kBlockM + ch * 8);
-          *reinterpret_cast<uint4*>(p.C + static_cast<size_t>(mm) * p.N + n_base + ch * 8) = val;
-        }
+      if (tid == 0) {
+        tma_store_2d(&tmC, s_c, n_base, 0);
+        bulk_commit_group();
       }
-      return group_sync(pbar, pphase, abort_flag);
+      store_pending = true;
+      return true;
     };
 
     for (int u = u_begin; u < u_end && ok;) {
@@ -1634,6 +1640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       first_segment = false;
       u = tu0 + kb1;
     }
+    if (store_pending && tid == 0) bulk_wait_all();  // the tile stores have completed
   }
 
   if (S > 1) {

@@ -245,6 +245,19 @@ bool encode_fp8_map_kblocks_grouped(CUtensorMap* map, const void* base, uint64_t
   return r == CUDA_SUCCESS;
 }
 
+// bf16 output map for the small-M kernel's tile stores: dims {N, M}, box {128, box_rows}, no swizzle
+// (its staging tile is row-major [token][128 columns]); rows past M and columns past N are clipped.
+bool encode_bf16_tile_store_map(CUtensorMap* map, void* base, uint64_t N, uint64_t M, uint32_t box_rows) {
+  cuuint64_t dims[2] = {N, M};
+  cuuint64_t strides[1] = {N * 2};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kBlockM), box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_fp8_map_2d(CUtensorMap* map, const void* base, uint64_t K, uint64_t rows, uint32_t box_rows) {
   cuuint64_t dims[2] = {K, rows};
   cuuint64_t strides[1] = {K};
@@ -736,7 +749,7 @@ fg_status run_swap_t(const Ctx* st, const void* A, const float* sfa, const void*
   p.static_b = (flags & FG_FLAG_STATIC_B) ? 1 : 0;
   if (p.n_tiles > kCounterCapacity) return FG_ERR_UNSUPPORTED;
 
-  CUtensorMap mW, mT;
+  CUtensorMap mW, mT, mC;
   if constexpr (KPS == 1) {
     if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
     if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
@@ -744,10 +757,11 @@ fg_status run_swap_t(const Ctx* st, const void* A, const float* sfa, const void*
     if (!encode_fp8_map_kblocks(&mW, B, K, N, kBlockM, KPS)) return FG_ERR_CUDA;
     if (!encode_fp8_map_kblocks(&mT, A, K, M, MP, KPS)) return FG_ERR_CUDA;
   }
+  if (!encode_bf16_tile_store_map(&mC, C, N, M, MP)) return FG_ERR_CUDA;
   const SwapChoice c = swap_choose<MP, KPS>(st->sms, p.n_tiles, p.num_kb);
   p.tile_aligned = c.tile_aligned;
   p.cluster = c.cluster;
-  void* args[3] = {&mW, &mT, &p};
+  void* args[4] = {&mW, &mT, &mC, &p};
   return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES, KPS>>(
       dim3(c.grid), swap_smem_bytes<MP, STAGES, KPS>(), stream, args, fg::kThreads, 0, c.cluster);
 }
@@ -844,15 +858,16 @@ fg_status run_swap_noalloc(const NoAllocDevice& d, const void* A, const float* s
   // wait may not have, so clear the ones this call uses (a memset, no allocation)
   if (cudaMemsetAsync(p.counters, 0, static_cast<size_t>(p.n_tiles) * sizeof(int), stream) != cudaSuccess)
     return FG_ERR_CUDA;
-  CUtensorMap mW, mT;
+  CUtensorMap mW, mT, mC;
   if (!encode_fp8_map_2d(&mW, B, K, N, kBlockM)) return FG_ERR_CUDA;
   if (!encode_fp8_map_2d(&mT, A, K, M, MP)) return FG_ERR_CUDA;
+  if (!encode_bf16_tile_store_map(&mC, C, N, M, MP)) return FG_ERR_CUDA;
   // the partial tiles (two per CTA) must fit in the array: that caps the grid, not the problem size
   const long long cap = static_cast<long long>(kNoAllocPartialBytes / (2 * MP * kBlockM * sizeof(float)));
   long long grid = static_cast<long long>(p.n_tiles) * p.num_kb;
   if (grid > d.sms) grid = d.sms;
   if (grid > cap) grid = cap;
-  void* args[3] = {&mW, &mT, &p};
+  void* args[4] = {&mW, &mT, &mC, &p};
   return launch<fg::fp8_gemm_swap_streamk_kernel<MP, STAGES>>(dim3(static_cast<unsigned>(grid)),
                                                                swap_smem_bytes<MP, STAGES>(), stream, args,
                                                                fg::kThreads);
