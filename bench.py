@@ -641,6 +641,8 @@ def run_ours(args, rank, world, local):
         fg.set_tile_n(args.tile_n)
     if args.stage_kblocks is not None:
         fg.set_stage_kblocks(args.stage_kblocks)
+    if args.tile_order is not None:
+        fg.set_tile_order(args.tile_order)
     stream = torch.cuda.Stream(device=dev)
     copy_gbs = box_copy_gbs(dev)
     name, wl = workload_list(args.workload, args.shape)
@@ -696,7 +698,8 @@ def run_ours(args, rank, world, local):
                            tiled_streamk="library default" if args.tiled_streamk is None else args.tiled_streamk,
                            swap_schedule="library default" if args.swap_schedule is None else args.swap_schedule,
                            tile_n="library default" if args.tile_n is None else args.tile_n,
-                           stage_kblocks="library default" if args.stage_kblocks is None else args.stage_kblocks),
+                           stage_kblocks="library default" if args.stage_kblocks is None else args.stage_kblocks,
+                           tile_order="library default" if args.tile_order is None else args.tile_order),
             "hbm_gbs": res["hbm_gbs"], "shapes": res["shapes"], "shapes_timing": res["shapes_timing"],
             "roofline": res["roofline"],
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS", "h2d_bytes_per_step": h2d,
@@ -760,6 +763,9 @@ def main():
     ap.add_argument("--stage-kblocks", type=int, default=None, choices=[0, 1, 2],
                     help="K blocks per ring stage of the small-M and CTA-pair kernels (fg_set_stage_kblocks): "
                          "0 automatic")
+    ap.add_argument("--tile-order", type=int, default=None, choices=[0, 1, 2],
+                    help="tile walk of the tiled family (fg_set_tile_order): 0 automatic, 1 m-block groups, "
+                         "2 n fastest")
     ap.add_argument("--record-traffic", default=None, metavar="CSV",
                     help="write profiles/traffic.json from an ncu launch list of this workload, then exit")
     args = ap.parse_args()

@@ -282,6 +282,14 @@ fg_status fg_jit_compile_check(int bn, int num_kb, int N, size_t* cubin_bytes);
  * identical.  Returns the previous value. */
 int fg_set_pair_promotion(int warpgroups);
 
+/* Tile walk of the tiled and CTA-pair kernels, process-wide: 0 (default) = automatic, 1 = groups of
+ * m-blocks whose A rows take at most 24 MB, m-block fastest inside a group (B streams through,
+ * re-read once per group), 2 = n-block fastest (each m-block's rows are read once while B stays
+ * in L2).  Automatic takes 2 when one group's B (N x K bytes) is at most 40 MB, else 1.  Other
+ * values are ignored.  Results are identical (each tile is computed the same way).  Returns the
+ * previous value. */
+int fg_set_tile_order(int order);
+
 /* The kernel and tile width a call of this shape takes on the current device under the
  * current settings, as kernel * 1000 + width: 1xxx the one-CTA tiled kernel, 3xxx the
  * CTA pair, 2000 the small-M swap-AB kernel (dense, M <= 128).  layout: 0 dense, 1

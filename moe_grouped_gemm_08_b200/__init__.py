@@ -72,6 +72,8 @@ def _declare(l: ctypes.CDLL) -> ctypes.CDLL:
     l.fg_set_dense_path.restype = _int
     l.fg_debug_set_stall.argtypes = [_int]
     l.fg_debug_set_stall.restype = _int
+    l.fg_set_tile_order.argtypes = [_int]
+    l.fg_set_tile_order.restype = _int
     l.fg_set_jit.argtypes = [_int]
     l.fg_set_jit.restype = _int
     l.fg_jit_cache_size.argtypes = []
@@ -168,6 +170,11 @@ def set_tile_n(bn: int) -> int:
     """Output tile width of the tiled / CTA-pair kernels: 0 automatic, or 128, 192, 256. Returns the
     old value."""
     return int(_lib.fg_set_tile_n(int(bn)))
+
+
+def set_tile_order(order: int) -> int:
+    """Tile walk of the tiled family: 0 automatic, 1 m-block groups (m fastest), 2 n fastest."""
+    return int(_lib.fg_set_tile_order(int(order)))
 
 
 def set_jit(enable: bool) -> int:

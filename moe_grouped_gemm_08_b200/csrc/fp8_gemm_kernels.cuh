@@ -90,6 +90,7 @@ struct TiledParams {
   int m_blocks; // ceil(M / 128)
   int n_blocks; // ceil(N / BN)
   int group_m;  // tile order: groups of group_m m-blocks, m-block fastest inside a group
+  int b_resident;  // 1: the walk keeps B in L2 (n-block fastest): A loads evict first, B loads last
   uint32_t fmt_bits;  // operand formats in instruction-descriptor position (0: both e4m3)
   float* ws;        // stream-K tail: 2 * gridDim.x partial tiles of 128 x BN fp32
   int* counters;    // stream-K tail: one per tile of the last partial wave, zero between launches
@@ -565,8 +566,10 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t issued = 0;
       bool ok = true;
-      const uint64_t pol_a = l2_policy_evict_last();   // A rows: re-read by every n-block of a group
-      const uint64_t pol_b = l2_policy_evict_first();  // B tiles: shared by the concurrent m-blocks only
+      // m-fastest groups: A rows are re-read by every n-block of a group, B tiles only by the
+      // concurrent m-blocks; n fastest: the other way round
+      const uint64_t pol_a = p.b_resident ? l2_policy_evict_first() : l2_policy_evict_last();
+      const uint64_t pol_b = p.b_resident ? l2_policy_evict_last() : l2_policy_evict_first();
       while (ok && tiled_next(plan, p.num_kb, cur, it)) {
         const TileInfo ti = tiled_tile<MODE>(p, s_prefix, live_mblocks, it.t, BN);
         if (!ti.live) continue;
@@ -972,8 +975,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<PW>::threa
       uint32_t issued = 0;
       bool ok = true;
       const uint32_t full_leader = mapa_shared(smem_addr(full), 0);
-      const uint64_t pol_a = l2_policy_evict_last();
-      const uint64_t pol_b = l2_policy_evict_first();
+      const uint64_t pol_a = p.b_resident ? l2_policy_evict_first() : l2_policy_evict_last();
+      const uint64_t pol_b = p.b_resident ? l2_policy_evict_last() : l2_policy_evict_first();
       for (int t = pair; t < num_tiles && ok; t += num_pairs) {
         const TileInfo ti = tiled_tile<MODE, PAIR_ROWS>(p, s_prefix, live_blocks, t, BN);
         const int ga = (MODE == kMasked) ? ti.g : 0;

@@ -64,7 +64,7 @@ std::atomic<uint64_t> g_launches{0};
 #define FG_TILED_STAGES 4
 #endif
 #ifndef FG_TILED_GROUP_MB
-#define FG_TILED_GROUP_MB 48  // L2 budget (MB) for the A rows of one group of m-blocks
+#define FG_TILED_GROUP_MB 24  // L2 budget (MB) for the A rows of one group of m-blocks
 #endif
 constexpr int kTiledBN = FG_TILED_BN;
 #ifndef FG_TILED_BN_MAX
@@ -84,6 +84,27 @@ constexpr int kPairStages = FG_PAIR_STAGES;
 
 // tile width of the tiled and pair kernels: 0 automatic, else forced (fg_set_tile_n)
 std::atomic<int> g_tile_n{0};
+// tile walk of the tiled family: 0 automatic, 1 groups of m-blocks (m fastest), 2 n fastest
+std::atomic<int> g_tile_order{0};
+
+// Tile walk (TiledParams::group_m): m-blocks in groups of group_m, m-block fastest inside a group;
+// group_m = 1 walks every n-block of an m-block before the next m-block (n fastest).  When one
+// group's (or the whole) B is small enough to stay in L2 (<= 40 MB), n fastest reads A once and B
+// once: the ~148 tiles in flight cover a few m-blocks and every n-block, so B stays resident while
+// A streams -- and in the grouped layouts consecutive m-blocks share an expert.  Larger B streams
+// through, with A in groups whose rows take at most FG_TILED_GROUP_MB of L2.  rows: rows per
+// m-block (128, or 256 for the CTA pair); mb_all: m-blocks in the walk.
+int tile_group_m(long long rows, int N, int K, long long mb_all, int* b_resident) {
+  constexpr long long kResidentB = 40ll << 20;
+  const int order = g_tile_order.load(std::memory_order_relaxed);
+  const long long b_bytes = static_cast<long long>(N) * K;
+  *b_resident = (order == 2 || (order == 0 && b_bytes <= kResidentB)) ? 1 : 0;
+  if (*b_resident) return 1;
+  long long gm = (static_cast<long long>(FG_TILED_GROUP_MB) << 20) / (rows * K);
+  if (gm < 1) gm = 1;
+  if (gm > mb_all) gm = mb_all;
+  return static_cast<int>(gm);
+}
 
 template <int BN>
 constexpr int tiled_stages() {
@@ -434,16 +455,8 @@ fg_status run_tiled(const Ctx* st, const void* A, const float* sfa, const void* 
   p.num_nb = (N + kBlockK - 1) / kBlockK;
   p.m_blocks = (M + kBlockM - 1) / kBlockM;
   p.n_blocks = (N + BN - 1) / BN;
-  // m-blocks per group of the tile walk: a group's A rows (128 * K bytes per m-block) should stay
-  // in L2 (126 MB) next to the streamed B tiles, so keep them within FG_TILED_GROUP_MB
-  {
-    const long long rows_bytes = static_cast<long long>(kBlockM) * K;
-    long long gm = (static_cast<long long>(FG_TILED_GROUP_MB) << 20) / rows_bytes;
-    if (gm < 1) gm = 1;
-    const long long mb_all = static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1);
-    if (gm > mb_all) gm = mb_all;
-    p.group_m = static_cast<int>(gm);
-  }
+  p.group_m = tile_group_m(kBlockM, N, K, static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1),
+                           &p.b_resident);
 
   CUtensorMap mA, mB, mC;
   const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;
@@ -536,14 +549,8 @@ fg_status run_pair(const Ctx* st, const void* A, const float* sfa, const void* B
   p.num_nb = (N + kBlockK - 1) / kBlockK;
   p.m_blocks = (M + 2 * kBlockM - 1) / (2 * kBlockM);  // 256-row blocks
   p.n_blocks = (N + BN - 1) / BN;
-  {
-    const long long rows_bytes = 2ll * kBlockM * K;
-    long long gm = (static_cast<long long>(FG_TILED_GROUP_MB) << 20) / rows_bytes;
-    if (gm < 1) gm = 1;
-    const long long mb_all = static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1);
-    if (gm > mb_all) gm = mb_all;
-    p.group_m = static_cast<int>(gm);
-  }
+  p.group_m = tile_group_m(2 * kBlockM, N, K, static_cast<long long>(p.m_blocks) * (MODE == fg::kMasked ? G : 1),
+                           &p.b_resident);
 
   CUtensorMap mA, mB, mC;
   const uint64_t groupsA = (MODE == fg::kMasked) ? static_cast<uint64_t>(G) : 1;
@@ -946,6 +953,11 @@ int fg_tile_plan(int layout, int M, int N, int K, int G) {
   if (layout == 0 && (path == 2 || (path == 0 && M <= kMaxSwapMP))) return 2000;
   const TilePlan t = tile_plan(layout, M, N, G, st->sms);
   return t.kernel * 1000 + t.bn;
+}
+
+int fg_set_tile_order(int order) {
+  if (order < 0 || order > 2) return g_tile_order.load();
+  return g_tile_order.exchange(order);
 }
 
 int fg_set_tile_n(int bn) {
