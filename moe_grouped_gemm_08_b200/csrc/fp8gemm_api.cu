@@ -146,7 +146,7 @@ constexpr int swap_stages() {
 template <int MP, int STAGES, int KPS = 1>
 constexpr size_t swap_smem_bytes() {
   return 1024 + static_cast<size_t>(STAGES) * KPS * (kBlockM + MP) * kBlockK + MP * kBlockM * 2 /*C staging*/ +
-         fg::kSwapScaleBytes /*combined scales*/ + 256 /*barriers*/;
+         fg::kSwapScaleBytes /*combined scales*/ + fg::kSwapBarrierBytes;
 }
 static_assert(swap_smem_bytes<32, swap_stages<32, 2>(), 2>() <= 227 * 1024, "swap kernel shared memory");
 static_assert(swap_smem_bytes<64, swap_stages<64, 2>(), 2>() <= 227 * 1024, "swap kernel shared memory");
