@@ -1394,23 +1394,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.debug_stall) mbar_wait(mma_done, 0, abort_flag, kWaitLimitNs);
       bool ok = true;
       for (int u = u_begin; u < u_end && ok; ++u) {
-        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
         const int nk = unit_kblocks(u);
         const uint32_t sw = smem_addr(smem + stage * STAGE_BYTES);
         if (KPS == 2 && nk == 2) {
           // one TMEM partial per K block; the two K blocks' MMAs are issued interleaved (K step j
           // of both, then step j + 1), so that their chains of dependent MMAs -- each accumulating
           // into its own buffer -- overlap in the tensor pipe instead of running one after the
-          // other (a decode step 5% faster at M = 64 than with the chains issued in turn)
+          // other (a decode step 5% faster at M = 64 than with the chains issued in turn).  The
+          // TMEM buffers are claimed and the descriptors formed before the wait for the data, so
+          // that only the MMAs follow its arrival.
           const uint32_t tb1 = tb + 1 == NUM_TBUF ? 0u : tb + 1;
           const uint32_t tph1 = tb + 1 == NUM_TBUF ? (tphase ^ 1u) : tphase;
           if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) break;
           if (!mbar_wait(&tempty[tb1], tph1 ^ 1u, abort_flag, kWaitLimitNs)) break;
-          tc_fence_after();
           const uint32_t d0 = tmem_base + tb * MP, d1 = tmem_base + tb1 * MP;
           const uint64_t a0 = smem_desc_k128_sw128(sw), a1 = smem_desc_k128_sw128(sw + W_BYTES);
           const uint64_t b0 = smem_desc_k128_sw128(sw + KPS * W_BYTES);
           const uint64_t b1 = smem_desc_k128_sw128(sw + KPS * W_BYTES + T_BYTES);
+          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
+          tc_fence_after();
 #pragma unroll
           for (int j = 0; j < kBlockK / 32; ++j) {
             mma_f8(d0, a0 + 2 * j, b0 + 2 * j, IDESC | p.fmt_bits, j > 0 ? 1u : 0u);
@@ -1422,6 +1424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (tb1 + 1 == NUM_TBUF || tb1 == 0) tphase ^= 1u;
           tb = tb1 + 1 == NUM_TBUF ? 0u : tb1 + 1;
         } else {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) break;
           for (int i = 0; i < nk; ++i) {  // one TMEM partial per K block
             if (!mbar_wait(&tempty[tb], tphase ^ 1u, abort_flag, kWaitLimitNs)) { ok = false; break; }
             tc_fence_after();
