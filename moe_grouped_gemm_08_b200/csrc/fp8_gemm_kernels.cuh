@@ -827,7 +827,9 @@ __global__ void __launch_bounds__(kTiledThreads, 1)
       ti = ti_next;
       have = have_next;
     }
-    if (stores_pending && lane == 0) bulk_wait_all();
+    // the staging areas must outlive the stores' reads of them; the global writes complete
+    // on their own before the grid completes
+    if (stores_pending && lane == 0) bulk_wait_read_all();
   }
 
   tc_fence_before();
@@ -1177,7 +1179,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<PW>::threa
       t = t_next;
       ti = ti_next;
     }
-    if (stores_pending && lane == 0) bulk_wait_all();
+    // the staging areas must outlive the stores' reads of them; the global writes complete
+    // on their own before the grid completes
+    if (stores_pending && lane == 0) bulk_wait_read_all();
   }
 
   tc_fence_before();
@@ -1213,34 +1217,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairShape<PW>::threa
 // until its peers have read it.  Every thread reaches both barriers, also after an abort.
 // Cluster split-K reduction of the swap kernel: this CTA (rank `rank` of S) sums weight rows
 // [rank 128/S, (rank+1) 128/S) of the tile over the S partials ([token][weight row] fp32 at shared
-// address `part` in every CTA of the cluster), in rank order, and stores them as bf16.  All S
-// loads of an element are issued before the sum.
+// address `part` in every CTA of the cluster), in rank order.  cluster_reduce_sum issues every
+// distributed-shared-memory load of the thread (ITEMS float4 from each of the S CTAs) before the
+// first sum, so that they take one round trip; cluster_reduce_write stores the sums as bf16.
 template <int S, int MP>
-__device__ __forceinline__ void cluster_reduce_store(const SwapParams& p, uint32_t part, int rank, int n_base,
-                                                     int tid) {
-  constexpr int R4 = kBlockM / S / 4;  // float4 per token row of this CTA's slice
-  constexpr int NPROMO = kPromoWarps * 32;
+struct ClusterReduce {
+  static constexpr int R4 = kBlockM / S / 4;  // float4 per token row of this CTA's slice
+  static constexpr int NPROMO = kPromoWarps * 32;
+  static constexpr int ITEMS = (MP * R4 + NPROMO - 1) / NPROMO;
+};
+
+template <int S, int MP>
+__device__ __forceinline__ void cluster_reduce_sum(const SwapParams& p, uint32_t part, int rank, int tid,
+                                                   float4 (&r)[ClusterReduce<S, MP>::ITEMS]) {
+  using CR = ClusterReduce<S, MP>;
   const int rows = p.M < MP ? p.M : MP;
-#pragma unroll 2
-  for (int f = tid; f < rows * R4; f += NPROMO) {
-    const int mm = f / R4;
-    const int col = rank * (kBlockM / S) + (f - mm * R4) * 4;
-    const uint32_t off = part + static_cast<uint32_t>((mm * kBlockM + col) * 4);
-    float4 v[S];
+  float4 v[CR::ITEMS][S];
 #pragma unroll
-    for (int q = 0; q < S; ++q) v[q] = ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)));
-    float4 r = v[0];
+  for (int it = 0; it < CR::ITEMS; ++it) {
+    const int f = tid + it * CR::NPROMO;
+    const int mm = f / CR::R4;
+    const int col = rank * (kBlockM / S) + (f - mm * CR::R4) * 4;
+    const uint32_t off = part + static_cast<uint32_t>((mm * kBlockM + col) * 4);
+#pragma unroll
+    for (int q = 0; q < S; ++q)
+      v[it][q] = f < rows * CR::R4 ? ld_dsmem_f4(mapa_shared(off, static_cast<uint32_t>(q)))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int it = 0; it < CR::ITEMS; ++it) {
+    r[it] = v[it][0];
 #pragma unroll
     for (int q = 1; q < S; ++q) {
-      r.x += v[q].x; r.y += v[q].y; r.z += v[q].z; r.w += v[q].w;
+      r[it].x += v[it][q].x; r[it].y += v[it][q].y; r[it].z += v[it][q].z; r[it].w += v[it][q].w;
     }
-    if (n_base + col < p.N) {  // N % 8 == 0, so the 4 columns are all inside
+  }
+}
+
+template <int S, int MP>
+__device__ __forceinline__ void cluster_reduce_write(const SwapParams& p, const float4 (&r)[ClusterReduce<S, MP>::ITEMS],
+                                                     int rank, int n_base, int tid) {
+  using CR = ClusterReduce<S, MP>;
+  const int rows = p.M < MP ? p.M : MP;
+#pragma unroll
+  for (int it = 0; it < CR::ITEMS; ++it) {
+    const int f = tid + it * CR::NPROMO;
+    const int mm = f / CR::R4;
+    const int col = rank * (kBlockM / S) + (f - mm * CR::R4) * 4;
+    if (f < rows * CR::R4 && n_base + col < p.N) {  // N % 8 == 0, so the 4 columns are all inside
       uint2 val;
-      val.x = pack_bf16x2(r.x, r.y);
-      val.y = pack_bf16x2(r.z, r.w);
+      val.x = pack_bf16x2(r[it].x, r[it].y);
+      val.y = pack_bf16x2(r[it].z, r[it].w);
       *reinterpret_cast<uint2*>(p.C + static_cast<size_t>(mm) * p.N + n_base + col) = val;
     }
   }
+}
+
+// All threads of the CTA: sum this CTA's slice over the cluster (promotion warps, unless the
+// kernel aborted), tell the cluster that this CTA has read its peers' shared memory, write the
+// slice, and wait until every peer has read this CTA's shared memory before it may exit.
+template <int S, int MP>
+__device__ __forceinline__ void cluster_reduce_tail(const SwapParams& p, uint32_t part, int rank, int n_base,
+                                                    bool reduce) {
+  const int tid = threadIdx.x;
+  float4 r[ClusterReduce<S, MP>::ITEMS];
+  if (reduce) cluster_reduce_sum<S, MP>(p, part, rank, tid, r);
+  __syncwarp();
+  cluster_arrive_relaxed();
+  if (reduce) cluster_reduce_write<S, MP>(p, r, rank, n_base, tid);
+  __syncwarp();
+  cluster_wait();
 }
 
 // KPS: K blocks per ring stage (and per unit of work).  KPS = 1 loads each K block's weight and
@@ -1578,6 +1624,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         FG_DCHECK(t < p.counter_cap && c_first <= static_cast<int>(blockIdx.x) &&
                       static_cast<int>(blockIdx.x) <= c_last && c_first >= 0 && c_last < P,
                   p.status);
+        // workspace slot of piece c: the tile's first CTA may hold it as the last segment of its
+        // range (slot 2c+1); every later CTA holds it as its first segment (slot 2c)
+        const int first_slot = sk_slot(c_first, P, U, tu0);
+        auto piece_slot = [&](int c) { return c == c_first ? first_slot : 2 * c; };
+        if (tu0 + kb1 >= u_end) {
+          // The CTA's last segment usually ends after the tile's other pieces, which their CTAs
+          // published early in their ranges: when the counter already holds all of them, this CTA
+          // is the last to arrive and sums the pieces without publishing its own (its ring is idle
+          // and holds its piece for the sum).  The sum runs in CTA order from zero, as on the
+          // other path, so the result is the same bits.
+          if (tid == 0) {
+            const int last = ld_relaxed_gpu(p.counters + t) == c_last - c_first;
+            if (last) {
+              fence_acq_rel_gpu();  // acquire the other CTAs' partials
+              p.counters[t] = 0;    // ready for the next launch
+            }
+            *s_last = last;
+          }
+          if (!group_sync(pbar, pphase, abort_flag)) { ok = false; break; }
+          if (*s_last) {
+            fence_proxy_async_smem();
+            float* own = reinterpret_cast<float*>(smem) + nl;
+#pragma unroll
+            for (int j = 0; j < COLS; ++j) own[(h * COLS + j) * kBlockM] = acc[j];
+            constexpr int PR = 1;  // pieces loaded per round (more spill registers)
+            float r[COLS];
+#pragma unroll
+            for (int j = 0; j < COLS; ++j) r[j] = 0.0f;
+#pragma unroll 1
+            for (int c0 = c_first; c0 <= c_last; c0 += PR) {
+              float v[PR][COLS];
+#pragma unroll
+              for (int k = 0; k < PR; ++k) {
+                const int c = c0 + k;
+                if (c == static_cast<int>(blockIdx.x)) {  // this CTA's piece, from shared memory
+#pragma unroll
+                  for (int j = 0; j < COLS; ++j) v[k][j] = own[(h * COLS + j) * kBlockM];
+                } else if (c <= c_last) {
+                  const float* src = p.ws + static_cast<size_t>(piece_slot(c)) * MP * kBlockM + nl;
+#pragma unroll
+                  for (int j = 0; j < COLS; ++j) v[k][j] = __ldcg(src + (h * COLS + j) * kBlockM);
+                }
+              }
+#pragma unroll
+              for (int k = 0; k < PR; ++k) {
+                if (c0 + k <= c_last) {
+#pragma unroll
+                  for (int j = 0; j < COLS; ++j) r[j] += v[k][j];
+                }
+              }
+            }
+            if (!store_tile(r, n_base)) { ok = false; break; }
+            first_segment = false;
+            u = tu0 + kb1;
+            continue;
+          }
+        }
         float* wp = p.ws + static_cast<size_t>(slot) * MP * kBlockM + nl;
 #pragma unroll
         for (int j = 0; j < COLS; ++j) wp[static_cast<size_t>(h * COLS + j) * kBlockM] = acc[j];
@@ -1598,10 +1701,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           float4 r[F4];
 #pragma unroll
           for (int i = 0; i < F4; ++i) r[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-          // workspace slot of piece c: the tile's first CTA may hold it as the last segment of its
-          // range (slot 2c+1); every later CTA holds it as its first segment (slot 2c)
-          const int first_slot = sk_slot(c_first, P, U, tu0);
-          auto piece_slot = [&](int c) { return c == c_first ? first_slot : 2 * c; };
           if (tu0 + kb1 >= u_end) {
             // The CTA's last segment: its ring is idle (every load consumed, every MMA done), so
             // the partials are pulled into it with cp.async, RING_SLOTS partials in flight, each
@@ -1674,22 +1773,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       first_segment = false;
       u = tu0 + kb1;
     }
-    if (store_pending && tid == 0) bulk_wait_all();  // the tile stores have completed
+    // the staging tile must outlive the last store's read of it; the global writes complete on
+    // their own before the grid completes
+    if (store_pending && tid == 0) bulk_wait_read_all();
   }
 
   if (S > 1) {
     // cluster split-K: sum rows [cl_rank R, (cl_rank + 1) R) of the tile over the S partials
     __syncwarp();
     cluster_sync_all();  // every CTA's partial is in its shared memory
-    if (warp < kPromoWarps && !*abort_flag) {
-      const uint32_t part = smem_addr(smem);
-      const int n_base = cl_tile * kBlockM;
-      if (S == 2) cluster_reduce_store<2, MP>(p, part, cl_rank, n_base, threadIdx.x);
-      else if (S == 4) cluster_reduce_store<4, MP>(p, part, cl_rank, n_base, threadIdx.x);
-      else cluster_reduce_store<8, MP>(p, part, cl_rank, n_base, threadIdx.x);
-    }
-    __syncwarp();
-    cluster_sync_all();  // no CTA leaves while a peer may still read its shared memory
+    const bool reduce = warp < kPromoWarps && !*abort_flag;
+    const uint32_t part = smem_addr(smem);
+    const int n_base = cl_tile * kBlockM;
+    if (S == 2) cluster_reduce_tail<2, MP>(p, part, cl_rank, n_base, reduce);
+    else if (S == 4) cluster_reduce_tail<4, MP>(p, part, cl_rank, n_base, reduce);
+    else cluster_reduce_tail<8, MP>(p, part, cl_rank, n_base, reduce);
   }
 
   tc_fence_before();

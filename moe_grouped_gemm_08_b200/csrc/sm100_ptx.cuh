@@ -153,10 +153,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
-// Wait until this thread's committed bulk stores have finished reading shared memory ...
+// Wait until this thread's committed bulk stores have finished reading shared memory (their global
+// writes complete on their own, at the latest before the grid completes).
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// ... or have completed entirely.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
@@ -252,6 +251,14 @@ __device__ __forceinline__ void cp_async_wait() {
 // CTA's, earlier global writes before later ones).
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
+// Relaxed load at GPU scope (a counter other CTAs update atomically); paired with
+// fence_acq_rel_gpu() on the reading side when its value is to order later loads.
+__device__ __forceinline__ int ld_relaxed_gpu(const int* ptr) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+  return v;
+}
+
 // Warpgroup register re-allocation (all four warps of a warpgroup execute it).
 template <int REGS>
 __device__ __forceinline__ void reg_alloc() {
@@ -286,6 +293,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
+
+// The two halves of a cluster barrier with no memory ordering on the arrival: for "this CTA has
+// finished reading its peers' shared memory" (the values read are already in registers), so the
+// arrival need not wait for this thread's outstanding global stores.  Warp-converged.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // 16-byte load from the shared memory of a CTA of the cluster (a shared::cluster address).
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
