@@ -62,6 +62,12 @@ def test_schedule_switches():
     assert old == 18  # default cost charged for publishing partial tiles, in K blocks
     assert fg.set_tiled_streamk(-5) == 0
     assert fg.set_tiled_streamk(old) == -1  # any negative value is stored as -1 (never split)
+    old = fg.set_tile_order(1)
+    assert old == 0  # automatic by default (by the bytes of one group's B)
+    assert fg.set_tile_order(2) == 1
+    assert fg.set_tile_order(3) == 2  # not a walk: ignored
+    assert fg.set_tile_order(-1) == 2
+    assert fg.set_tile_order(old) == 2
 
 
 def test_swap_plan_without_device_state():
